@@ -1,0 +1,486 @@
+"""Benchmark of the fused compressed-state AdamW step (libfo, sm_100a).
+
+Default workload: the Llama-3.1-8B parameter list (291 tensors, 8,030,261,248
+parameters), bf16 + 8-bit ECC masters, 8-bit companded m / v, bf16 Student-t
+gradients; one step = one multi-tensor fo_adamw_step launch over all 291
+tensors.  Inputs are resident in HBM before timing; one step moves ~98 GB,
+far above the 126 MB L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+    python bench.py --impl reference ...     # the CPU oracle, timed on host cores
+
+Prints one JSON line (rank 0).  Multi-GPU: one process per GPU (torchrun),
+each rank steps its own parameter shard of the same shape (weak scaling, no
+data-path collective); time = max over ranks of the device-event time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused AdamW step Gparams/s and achieved HBM GB/s vs B200 peak"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="fo", choices=["fo", "reference"])
+    ap.add_argument("--config", default="llama3.1-8b")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-params", type=int, default=1 << 24)
+    ap.add_argument("--launch-mode", default="multi", choices=["multi", "release"])
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes (what the method must move)
+
+def algorithmic_bytes(wl) -> int:
+    """Bytes one step must read + write: downcast weights (r+w), ECC (r+w),
+    gradient (r), momentum codes (r+w) and scales (r+w), variance codes and
+    scales (r+w, AdamW only)."""
+    wb = 2
+    eb = wl.ecc_bits // 8
+    total = 0
+    for t in wl.tensors:
+        n = t.numel
+        ng = (n + 31) // 32
+        rd = n * (wb + eb + 2 + 1) + 2 * ng
+        wr = n * (wb + eb + 1) + 2 * ng
+        if wl.optimizer == "adamw":
+            rd += n + 2 * ng
+            wr += n + 2 * ng
+        total += rd + wr
+    return total
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("fo_codec.cuh", "fo_kernels.cuh", "fo_api.cu"):
+        with open(os.path.join(ROOT, "bit_states_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profile(config: str):
+    """dram bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(config)
+    if not e or e.get("kernel_source_sha") != kernel_source_sha():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        # samples under load: power above the idle level
+        load = [s for s, p in zip(sm, pw) if p > 200.0] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(load),
+                "power_w_max": max(pw) if pw else None}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline; also the reference arm)
+
+def cpu_sample(wl, n_params: int, rank_seed: int = 0):
+    """A bounded sample of the workload for the oracle: whole groups drawn
+    uniformly from every tensor in proportion to its size."""
+    import oracle
+
+    rng = np.random.default_rng(1234 + rank_seed)
+    total = wl.numel
+    parts = []
+    for ti, t in enumerate(wl.tensors):
+        ng = (t.numel + 31) // 32
+        k = max(1, int(round(n_params / 32 * t.numel / total)))
+        k = min(k, ng)
+        g = np.sort(rng.choice(ng, size=k, replace=False)) if k < ng else np.arange(ng)
+        g = g[32 * g + 32 <= t.numel] if (32 * g + 32 > t.numel).any() and g.size > 1 else g
+        idx = (32 * g[:, None] + np.arange(32)[None, :]).ravel()
+        idx = idx[idx < t.numel]
+        x = wl.master_values(ti, idx)
+        gb = wl.grad_bits(ti, 1, idx)
+        parts.append((x, gb))
+    x = np.concatenate([p[0] for p in parts])
+    gb = np.concatenate([p[1] for p in parts])
+    w, e = oracle.encode_master(x, 0 if wl.w_dtype == "bf16" else 1, wl.ecc_bits, threads=os.cpu_count() or 1)
+    return w, e, gb
+
+
+def time_oracle(wl, n_params: int, steps: int, warmup: int, threads: int):
+    import oracle
+
+    w, e, gb = cpu_sample(wl, n_params)
+    st = oracle.State.zeros_like_master(w, e, adam=(wl.optimizer == "adamw"))
+    wdt = 0 if wl.w_dtype == "bf16" else 1
+    gdt = 0 if wl.grad_dtype == "bf16" else 1
+
+    def one(t):
+        if wl.optimizer == "adamw":
+            oracle.adamw_step(st, gb, **wl.hparams, step=t, wdt=wdt, gdt=gdt, ecc_bits=wl.ecc_bits,
+                              threads=threads)
+        else:
+            h = wl.hparams
+            oracle.sgdm_step(st, gb, lr=h["lr"], momentum=h["momentum"], dampening=h["dampening"],
+                             weight_decay=h["weight_decay"], nesterov=bool(h["nesterov"]), step=t, wdt=wdt,
+                             gdt=gdt, ecc_bits=wl.ecc_bits, threads=threads)
+
+    for t in range(1, warmup + 1):
+        one(t)
+    t0 = time.perf_counter()
+    for k in range(steps):
+        one(warmup + 1 + k)
+    dt = time.perf_counter() - t0
+    n = w.size
+    return n * steps / dt / 1e9, dt, n
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    from workloads import workload
+
+    wl = workload(args.config)
+    threads = os.cpu_count() or 1
+    # each step is a bounded sample of the workload sized to keep the whole
+    # run within a few minutes of host time
+    n_params = min(args.cpu_sample_params, 1 << 24)
+    value, dt, n = time_oracle(wl, n_params, args.steps if args.steps <= 20 else 20, min(args.warmup, 3), threads)
+    steps = args.steps if args.steps <= 20 else 20
+    sample = f"{n} params per step (whole 32-groups drawn from all {len(wl.tensors)} tensors of {wl.name}), " \
+             f"AdamW step 1.., {threads} host threads"
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "Gparams/s",
+            "n_gpus": args.gpus, "steps": steps, "warmup": min(args.warmup, 3),
+            "ms_per_step": round(dt / steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": wl.name, "params": wl.numel, "sampled_params_per_step": n,
+                       "optimizer": wl.optimizer, "format": f"{wl.w_dtype}+ecc{wl.ecc_bits}"},
+            "cpu_baseline": {"value": round(value, 6), "unit": "Gparams/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "Gparams/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+
+    if not torch.cuda.is_available():
+        print(json.dumps({"metric": METRIC, "error": "no CUDA device"}), flush=True)
+        return 1
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+
+    from bit_states_b200 import build as fobuild
+    from bit_states_b200 import fo
+    from bit_states_b200.state import CompressedParams
+    from workloads import device as wdev
+    from workloads import workload
+
+    fobuild.build()
+    wdev.build()
+    fo.load()
+
+    wl = workload(args.config)
+    wl.seed = rank  # each rank steps its own shard (same shapes, its own values)
+    adam = wl.optimizer == "adamw"
+    dev = torch.device("cuda", local)
+    P = CompressedParams([t.numel for t in wl.tensors], dev, adam=adam, ecc_bits=wl.ecc_bits,
+                         w_dtype=wl.w_dtype)
+    buf = torch.empty(max(t.numel for t in wl.tensors), dtype=torch.float32, device=dev)
+    for ti, t in enumerate(wl.tensors):
+        x = buf[:t.numel]
+        wdev.master_f32(wl, ti, x)
+        P.encode_from(ti, x)
+    del buf
+    garena = torch.empty(P.total, dtype=torch.int16, device=dev)
+    gviews = [garena[o:o + n] for o, n in zip(P.offsets, P.numels)]
+    for ti, v in enumerate(gviews):
+        wdev.grad_16(wl, ti, 1, v)
+    torch.cuda.synchronize()
+
+    fmt = fo.make_format(wl.w_dtype, wl.grad_dtype, wl.ecc_bits)
+    h = wl.hparams
+    stream = torch.cuda.current_stream()
+    descs = fo.descriptors(P.states, gviews)
+    order = list(range(len(wl.tensors)))[::-1]
+    single = [fo.descriptors([P.states[i]], [gviews[i]]) for i in order]
+    launches_per_step = 1 if args.launch_mode == "multi" else len(order)
+    if args.launch_mode == "multi" and len(wl.tensors) > 384:
+        launches_per_step = (len(wl.tensors) + 383) // 384
+
+    def do_step(t):
+        if adam:
+            hp = fo.fo_adamw_hparams(h["lr"], h["beta1"], h["beta2"], h["eps"], h["weight_decay"], t)
+            if args.launch_mode == "multi":
+                fo.fo_adamw_step(descs, len(P.states), fmt, hp, stream)
+            else:
+                for d in single:
+                    fo.fo_adamw_step(d, 1, fmt, hp, stream)
+        else:
+            hp = fo.fo_sgdm_hparams(h["lr"], h["momentum"], h["dampening"], h["weight_decay"],
+                                    int(h["nesterov"]), t)
+            if args.launch_mode == "multi":
+                fo.fo_sgdm_step(descs, len(P.states), fmt, hp, stream)
+            else:
+                for d in single:
+                    fo.fo_sgdm_step(d, 1, fmt, hp, stream)
+
+    t = 0
+    for _ in range(args.warmup):
+        t += 1
+        do_step(t)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+
+    gpu_id = "0"
+    try:
+        props = torch.cuda.get_device_properties(local)
+        gpu_id = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+    except Exception:
+        gpu_id = os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[local] if "CUDA_VISIBLE_DEVICES" in os.environ else str(local)
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+
+    K = args.steps
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    for k in range(K):
+        t += 1
+        ev_s[k].record(stream)
+        do_step(t)
+        ev_e[k].record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clocks = sampler.stop()
+    total_ms = ev_s[0].elapsed_time(ev_e[K - 1])
+    per_launch_ms = statistics.mean(ev_s[k].elapsed_time(ev_e[k]) for k in range(K))
+    if dist:
+        tt = torch.tensor([total_ms, per_launch_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms, per_launch_ms = float(tt[0]), float(tt[1])
+
+    n_params = wl.numel
+    value = world * n_params * K / (total_ms / 1e3) / 1e9
+    abytes = algorithmic_bytes(wl)
+    peak, peak_kind = measured_peaks()
+    achieved = abytes / (per_launch_ms / 1e3) / 1e9 if launches_per_step == 1 else abytes / (per_launch_ms / 1e3) / 1e9
+    traffic = traffic_from_profile(args.config) if launches_per_step == 1 else None
+
+    # ---- end to end through the public API with host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, wl, P, fmt, dev, dist, world, torch, fo)
+
+    # ---- CPU oracle baseline (rank 0, N = 1) ----
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = os.cpu_count() or 1
+        v, dt, n = time_oracle(wl, args.cpu_sample_params, 1, 1, threads)
+        cpu = {"value": round(v, 6), "unit": "Gparams/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n} params (whole 32-groups drawn from all {len(wl.tensors)} tensors), one "
+                         f"{wl.optimizer} step after one warm step, {threads} host threads, {dt:.2f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": "Gparams/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": round(total_ms / K, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"{wl.name}: {len(wl.tensors)} tensors, {n_params} params per GPU, "
+                                   f"{wl.optimizer} {wl.w_dtype}+ecc{wl.ecc_bits}, int8/uint8 companded states",
+                       "launch": "one multi-tensor launch per step" if args.launch_mode == "multi" else
+                                 f"{len(order)} per-tensor launches per step (gradient release order)",
+                       "l2": "inputs larger than L2 (%.1f GB per step vs 126 MB)" % (abytes / 1e9),
+                       "parallelism": f"weak-scaling shards x{world}, no data-path collective"},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": traffic,
+                         "peak_kind": peak_kind, "algorithmic_bytes_per_launch": abytes,
+                         "kernel": "fo::step_kernel"},
+            "clocks": clocks,
+            "gpu_launches": K * launches_per_step,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def run_e2e(args, wl, P, fmt, dev, dist, world, torch, fo):
+    """Same metric through the public API with host buffers: every step
+    copies each tensor's bf16 gradient from pinned host memory and reads the
+    updated downcast weights back to pinned host memory, per tensor in
+    gradient-release order, copies overlapped with the step kernels."""
+    from bit_states_b200.state import CompressedAdamW
+
+    if wl.optimizer != "adamw":
+        return None
+    opt = CompressedAdamW(P, lr=wl.hparams["lr"], betas=(wl.hparams["beta1"], wl.hparams["beta2"]),
+                          eps=wl.hparams["eps"], weight_decay=wl.hparams["weight_decay"], grad_dtype=wl.grad_dtype)
+    from workloads import device as wdev
+
+    big = max(P.numels)
+    stage = [torch.empty(big, dtype=torch.int16, device=dev) for _ in range(2)]
+    # host gradients: the largest tensor's synthetic gradient, reused as the
+    # source of every tensor's copy (the bytes moved are the full list's)
+    wdev.grad_16(wl, int(np.argmax(P.numels)), 1, stage[0])
+    host_g = torch.empty(big, dtype=torch.int16, pin_memory=True)
+    host_g.copy_(stage[0])
+    host_w = torch.empty(big, dtype=torch.int16, pin_memory=True)
+    s_in = torch.cuda.Stream(dev)
+    s_out = torch.cuda.Stream(dev)
+    comp = torch.cuda.current_stream(dev)
+    order = list(range(len(P.numels)))[::-1]
+    h2d = sum(P.numels) * 2
+    d2h = sum(P.numels) * 2
+
+    def one_step(t):
+        done = [None, None]
+        for j, ti in enumerate(order):
+            n = P.numels[ti]
+            b = j % 2
+            with torch.cuda.stream(s_in):
+                if done[b] is not None:
+                    s_in.wait_event(done[b])
+                stage[b][:n].copy_(host_g[:n], non_blocking=True)
+                ev_in = torch.cuda.Event()
+                ev_in.record(s_in)
+            comp.wait_event(ev_in)
+            opt.step_tensor(ti, stage[b][:n], t, comp)
+            ev_done = torch.cuda.Event()
+            ev_done.record(comp)
+            done[b] = ev_done
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done)
+                host_w[:n].copy_(P.states[ti].w, non_blocking=True)
+        comp.wait_stream(s_out)
+        comp.wait_stream(s_in)
+
+    t0 = 10_000
+    one_step(t0)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    K = args.e2e_steps
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(comp)
+    for k in range(K):
+        one_step(t0 + 1 + k)
+    e1.record(comp)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if dist:
+        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt[0])
+    value = world * sum(P.numels) * K / (ms / 1e3) / 1e9
+    return {"value": round(value, 3), "unit": "Gparams/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(ms / K, 3), "steps": K,
+            "how": "per tensor: pinned-host bf16 grad -> device (copy stream), fo_adamw_step, updated bf16 "
+                   "weights -> pinned host (copy stream); double-buffered, overlapped"}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,325 @@
+// fo_api.cu - host side of libfo: argument validation, the binary32 host
+// scalars of one step, packing of the multi-tensor descriptor table into
+// kernel parameters, and launches.  See include/fo.h for the contract.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include <cuda_runtime.h>
+
+#include "fo.h"
+#include "fo_kernels.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+fo_status fail(fo_status s, const std::string& msg)
+{
+    g_last_error = msg;
+    return s;
+}
+
+fo_status cuda_fail(cudaError_t e, const char* where)
+{
+    return fail(FO_ERR_CUDA, std::string(where) + ": " + cudaGetErrorName(e) + " (" +
+                                 cudaGetErrorString(e) + ")");
+}
+
+// ---- per-device launch constants -------------------------------------------
+
+constexpr int kMaxDevices = 64;
+std::once_flag g_dev_once[kMaxDevices];
+int g_sm_count[kMaxDevices];
+
+fo_status device_sms(int* sms)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(FO_ERR_CUDA, "device ordinal out of range");
+    std::call_once(g_dev_once[dev], [dev] {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 0;
+        g_sm_count[dev] = n;
+    });
+    if (g_sm_count[dev] <= 0) return fail(FO_ERR_CUDA, "could not query the SM count");
+    *sms = g_sm_count[dev];
+    return FO_OK;
+}
+
+// ---- validation ------------------------------------------------------------
+
+bool aligned(const void* p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
+
+fo_status check_format(const fo_format& f)
+{
+    if ((f.w_dtype != FO_DT_BF16 && f.w_dtype != FO_DT_FP16) ||
+        (f.grad_dtype != FO_DT_BF16 && f.grad_dtype != FO_DT_FP16))
+        return fail(FO_ERR_UNSUPPORTED, "w_dtype / grad_dtype must be FO_DT_BF16 or FO_DT_FP16");
+    if (f.ecc_bits != 8 && f.ecc_bits != 16)
+        return fail(FO_ERR_UNSUPPORTED, "ecc_bits must be 8 or 16");
+    return FO_OK;
+}
+
+fo_status check_tensors(const fo_tensor* t, int n, const fo_format& f, bool adam)
+{
+    if (n < 0) return fail(FO_ERR_INVALID_ARG, "n_tensors < 0");
+    if (n > FO_MAX_TENSORS_PER_CALL) return fail(FO_ERR_TOO_MANY_TENSORS, "n_tensors too large");
+    if (n > 0 && t == nullptr) return fail(FO_ERR_INVALID_ARG, "tensor array is NULL");
+    for (int i = 0; i < n; i++) {
+        const fo_tensor& x = t[i];
+        char where[64];
+        snprintf(where, sizeof where, "tensor %d: ", i);
+        if (x.numel < 0) return fail(FO_ERR_INVALID_ARG, std::string(where) + "numel < 0");
+        if (x.numel == 0) continue;
+        if (!x.w || !x.ecc || !x.grad || !x.m_q || !x.m_scale)
+            return fail(FO_ERR_INVALID_ARG, std::string(where) + "NULL w / ecc / grad / m_q / m_scale");
+        if (adam && (!x.v_q || !x.v_scale))
+            return fail(FO_ERR_INVALID_ARG, std::string(where) + "NULL v_q / v_scale");
+        if (!aligned(x.w, 2) || !aligned(x.grad, 2) || !aligned(x.m_scale, 2) ||
+            (adam && !aligned(x.v_scale, 2)) || (f.ecc_bits == 16 && !aligned(x.ecc, 2)))
+            return fail(FO_ERR_ALIGNMENT, std::string(where) + "16-bit array not 2-byte aligned");
+    }
+    return FO_OK;
+}
+
+// ---- launch of one step over a tensor list -----------------------------------
+
+using StepKernel = void (*)(const fo::StepParams);
+
+template <int KIND>
+StepKernel pick_step(const fo_format& f)
+{
+#define FO_PICK(W, G, N)                                                                  \
+    if (f.w_dtype == W && f.grad_dtype == G && f.ecc_bits == N) return fo::step_kernel<W, G, N, KIND>;
+    FO_PICK(0, 0, 8) FO_PICK(0, 1, 8) FO_PICK(1, 0, 8) FO_PICK(1, 1, 8)
+    FO_PICK(0, 0, 16) FO_PICK(0, 1, 16) FO_PICK(1, 0, 16) FO_PICK(1, 1, 16)
+#undef FO_PICK
+    return nullptr;
+}
+
+struct OccCache {
+    std::mutex mu;
+    const void* fn[64] = {};
+    int blocks[64] = {};
+    int n = 0;
+} g_occ;
+
+int blocks_per_sm(StepKernel k)
+{
+    std::lock_guard<std::mutex> lock(g_occ.mu);
+    for (int i = 0; i < g_occ.n; i++)
+        if (g_occ.fn[i] == (const void*)k) return g_occ.blocks[i];
+    int b = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, k, fo::kThreads, 0) != cudaSuccess || b < 1)
+        b = 1;
+    if (g_occ.n < 64) {
+        g_occ.fn[g_occ.n] = (const void*)k;
+        g_occ.blocks[g_occ.n] = b;
+        g_occ.n++;
+    }
+    return b;
+}
+
+fo_status launch_step(StepKernel k, const fo::Scalars& sc, const fo_tensor* t, int n,
+                      cudaStream_t stream)
+{
+    bool any = false;
+    for (int j = 0; j < n && !any; j++) any = t[j].numel > 0;
+    if (!any) return FO_OK;
+    int sms = 0;
+    fo_status st = device_sms(&sms);
+    if (st != FO_OK) return st;
+    const int bps = blocks_per_sm(k);
+    // kernel parameters are copied at launch, so one block of host memory
+    // per thread serves every launch
+    thread_local fo::StepParams P;
+    int i = 0;
+    while (i < n) {
+        std::memset(&P, 0, offsetof(fo::StepParams, t));
+        P.sc = sc;
+        int m = 0;
+        int64_t chunks = 0;
+        P.chunk_start[0] = 0;
+        for (; i < n && m < fo::kMaxTensorsPerLaunch; i++) {
+            const fo_tensor& x = t[i];
+            if (x.numel == 0) continue;
+            fo::TensorDesc& d = P.t[m];
+            d.w = x.w;
+            d.ecc = x.ecc;
+            d.grad = x.grad;
+            d.mq = x.m_q;
+            d.ms = x.m_scale;
+            d.vq = x.v_q;
+            d.vs = x.v_scale;
+            d.numel = x.numel;
+            chunks += (x.numel + fo::kChunk - 1) / fo::kChunk;
+            P.chunk_start[++m] = chunks;
+        }
+        if (m == 0) break;
+        P.n_tensors = m;
+        P.total_chunks = chunks;
+        // a sentinel past the last tensor keeps the device-side walk bounded
+        for (int j = m + 1; j <= fo::kMaxTensorsPerLaunch; j++) P.chunk_start[j] = INT64_MAX;
+        const int64_t warps_per_block = fo::kThreads / 32;
+        int64_t grid = (chunks + warps_per_block - 1) / warps_per_block;
+        const int64_t cap = (int64_t)sms * bps;
+        if (grid > cap) grid = cap;
+        k<<<(unsigned)grid, fo::kThreads, 0, stream>>>(P);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "step kernel launch");
+    }
+    return FO_OK;
+}
+
+bool is_finite(double v) { return std::isfinite(v); }
+
+int64_t grid_for(int64_t n, int sms)
+{
+    int64_t g = (n + fo::kThreads - 1) / fo::kThreads;
+    const int64_t cap = (int64_t)sms * 8;
+    if (g > cap) g = cap;
+    return g < 1 ? 1 : g;
+}
+
+}  // namespace
+
+extern "C" {
+
+fo_status fo_adamw_step(const fo_tensor* t, int n_tensors, fo_format f, const fo_adamw_hparams* h,
+                        void* stream)
+{
+    g_last_error.clear();
+    fo_status st = check_format(f);
+    if (st != FO_OK) return st;
+    if (!h) return fail(FO_ERR_INVALID_ARG, "hyper-parameters are NULL");
+    if (!is_finite(h->lr) || !is_finite(h->eps) || !is_finite(h->weight_decay))
+        return fail(FO_ERR_INVALID_ARG, "lr / eps / weight_decay must be finite");
+    if (!(h->beta1 >= 0.0 && h->beta1 < 1.0) || !(h->beta2 >= 0.0 && h->beta2 < 1.0))
+        return fail(FO_ERR_INVALID_ARG, "betas must lie in [0, 1)");
+    if (h->step < 1) return fail(FO_ERR_INVALID_ARG, "step must be >= 1");
+    st = check_tensors(t, n_tensors, f, true);
+    if (st != FO_OK) return st;
+    if (n_tensors == 0) return FO_OK;
+    // host scalars: binary64, each rounded once to binary32
+    const double bc1 = 1.0 - std::pow(h->beta1, (double)h->step);
+    const double bc2 = 1.0 - std::pow(h->beta2, (double)h->step);
+    fo::Scalars sc;
+    sc.s[0] = (float)h->beta1;
+    sc.s[1] = (float)h->beta2;
+    sc.s[2] = (float)(1.0 - h->beta1);
+    sc.s[3] = (float)(1.0 - h->beta2);
+    sc.s[4] = (float)(h->lr / bc1);
+    sc.s[5] = (float)(1.0 / std::sqrt(bc2));
+    sc.s[6] = (float)h->eps;
+    sc.s[7] = (float)(1.0 - h->lr * h->weight_decay);
+    StepKernel k = pick_step<fo::kAdamW>(f);
+    if (!k) return fail(FO_ERR_UNSUPPORTED, "format not provided");
+    return launch_step(k, sc, t, n_tensors, (cudaStream_t)stream);
+}
+
+fo_status fo_sgdm_step(const fo_tensor* t, int n_tensors, fo_format f, const fo_sgdm_hparams* h,
+                       void* stream)
+{
+    g_last_error.clear();
+    fo_status st = check_format(f);
+    if (st != FO_OK) return st;
+    if (!h) return fail(FO_ERR_INVALID_ARG, "hyper-parameters are NULL");
+    if (!is_finite(h->lr) || !is_finite(h->weight_decay))
+        return fail(FO_ERR_INVALID_ARG, "lr / weight_decay must be finite");
+    if (!(h->momentum >= 0.0 && h->momentum <= 1.0) || !(h->dampening >= 0.0 && h->dampening <= 1.0))
+        return fail(FO_ERR_INVALID_ARG, "momentum / dampening must lie in [0, 1]");
+    if (h->step < 1) return fail(FO_ERR_INVALID_ARG, "step must be >= 1");
+    st = check_tensors(t, n_tensors, f, false);
+    if (st != FO_OK) return st;
+    if (n_tensors == 0) return FO_OK;
+    fo::Scalars sc;
+    sc.s[0] = (float)h->lr;
+    sc.s[1] = (float)h->momentum;
+    sc.s[2] = (float)(1.0 - h->dampening);
+    sc.s[3] = (float)h->weight_decay;
+    sc.s[4] = h->nesterov ? 1.0f : 0.0f;
+    sc.s[5] = h->step == 1 ? 1.0f : 0.0f;
+    sc.s[6] = 0.0f;
+    sc.s[7] = 0.0f;
+    StepKernel k = pick_step<fo::kSGDM>(f);
+    if (!k) return fail(FO_ERR_UNSUPPORTED, "format not provided");
+    return launch_step(k, sc, t, n_tensors, (cudaStream_t)stream);
+}
+
+fo_status fo_encode_master(const float* x32, void* w, void* ecc, int64_t n, fo_format f, void* stream)
+{
+    g_last_error.clear();
+    fo_status st = check_format(f);
+    if (st != FO_OK) return st;
+    if (n < 0) return fail(FO_ERR_INVALID_ARG, "n < 0");
+    if (n == 0) return FO_OK;
+    if (!x32 || !w || !ecc) return fail(FO_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned(x32, 4) || !aligned(w, 2) || (f.ecc_bits == 16 && !aligned(ecc, 2)))
+        return fail(FO_ERR_ALIGNMENT, "misaligned array");
+    int sms = 0;
+    st = device_sms(&sms);
+    if (st != FO_OK) return st;
+    const unsigned grid = (unsigned)grid_for(n, sms);
+    cudaStream_t s = (cudaStream_t)stream;
+    const bool bf = f.w_dtype == FO_DT_BF16;
+    if (f.ecc_bits == 8) {
+        if (bf) fo::encode_master_kernel<0, 8><<<grid, fo::kThreads, 0, s>>>(x32, w, ecc, n);
+        else fo::encode_master_kernel<1, 8><<<grid, fo::kThreads, 0, s>>>(x32, w, ecc, n);
+    } else {
+        if (bf) fo::encode_master_kernel<0, 16><<<grid, fo::kThreads, 0, s>>>(x32, w, ecc, n);
+        else fo::encode_master_kernel<1, 16><<<grid, fo::kThreads, 0, s>>>(x32, w, ecc, n);
+    }
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? FO_OK : cuda_fail(e, "encode kernel launch");
+}
+
+fo_status fo_decode_master(const void* w, const void* ecc, float* x32, int64_t n, fo_format f,
+                           void* stream)
+{
+    g_last_error.clear();
+    fo_status st = check_format(f);
+    if (st != FO_OK) return st;
+    if (n < 0) return fail(FO_ERR_INVALID_ARG, "n < 0");
+    if (n == 0) return FO_OK;
+    if (!x32 || !w || !ecc) return fail(FO_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned(x32, 4) || !aligned(w, 2) || (f.ecc_bits == 16 && !aligned(ecc, 2)))
+        return fail(FO_ERR_ALIGNMENT, "misaligned array");
+    int sms = 0;
+    st = device_sms(&sms);
+    if (st != FO_OK) return st;
+    const unsigned grid = (unsigned)grid_for(n, sms);
+    cudaStream_t s = (cudaStream_t)stream;
+    const bool bf = f.w_dtype == FO_DT_BF16;
+    if (f.ecc_bits == 8) {
+        if (bf) fo::decode_master_kernel<0, 8><<<grid, fo::kThreads, 0, s>>>(w, ecc, x32, n);
+        else fo::decode_master_kernel<1, 8><<<grid, fo::kThreads, 0, s>>>(w, ecc, x32, n);
+    } else {
+        if (bf) fo::decode_master_kernel<0, 16><<<grid, fo::kThreads, 0, s>>>(w, ecc, x32, n);
+        else fo::decode_master_kernel<1, 16><<<grid, fo::kThreads, 0, s>>>(w, ecc, x32, n);
+    }
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? FO_OK : cuda_fail(e, "decode kernel launch");
+}
+
+const char* fo_status_string(fo_status s)
+{
+    switch (s) {
+    case FO_OK: return "FO_OK";
+    case FO_ERR_INVALID_ARG: return "FO_ERR_INVALID_ARG";
+    case FO_ERR_UNSUPPORTED: return "FO_ERR_UNSUPPORTED";
+    case FO_ERR_ALIGNMENT: return "FO_ERR_ALIGNMENT";
+    case FO_ERR_TOO_MANY_TENSORS: return "FO_ERR_TOO_MANY_TENSORS";
+    case FO_ERR_CUDA: return "FO_ERR_CUDA";
+    }
+    return "unknown fo_status";
+}
+
+const char* fo_last_error(void) { return g_last_error.c_str(); }
+
+int fo_version(void) { return 100; }
+
+}  // extern "C"

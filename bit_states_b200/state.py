@@ -1,0 +1,130 @@
+"""Compressed optimizer state of a parameter list, in device memory.
+
+Buffers are allocated with torch (plumbing only) as one arena per stream of
+bytes: downcast weights, ECC codes, momentum codes + scales, variance codes +
+scales.  Each tensor's slice starts on a multiple of 512 elements, so every
+array of every tensor is aligned for the kernels' 256-bit accesses.  All
+arithmetic (encode, step, decode) runs in libfo's kernels.
+"""
+from __future__ import annotations
+
+from typing import List, Sequence
+
+from . import fo
+
+ALIGN_ELEMS = 512
+
+
+def _round_up(n: int, a: int) -> int:
+    return (n + a - 1) // a * a
+
+
+class CompressedParams:
+    """Arena of the compressed state of ``numels`` parameters."""
+
+    def __init__(self, numels: Sequence[int], device, adam: bool = True, ecc_bits: int = 8,
+                 w_dtype: str = "bf16"):
+        import torch
+
+        self.numels = [int(n) for n in numels]
+        self.adam = adam
+        self.ecc_bits = ecc_bits
+        self.w_dtype = w_dtype
+        self.offsets: List[int] = []
+        self.goffsets: List[int] = []
+        off = goff = 0
+        for n in self.numels:
+            self.offsets.append(off)
+            self.goffsets.append(goff)
+            off += _round_up(max(n, 1), ALIGN_ELEMS)
+            goff += _round_up((n + 31) // 32, 16)
+        self.total = off
+        self.gtotal = goff
+        edt = torch.int8 if ecc_bits == 8 else torch.int16
+        self.w = torch.zeros(self.total, dtype=torch.int16, device=device)
+        self.ecc = torch.zeros(self.total, dtype=edt, device=device)
+        self.m_q = torch.zeros(self.total, dtype=torch.int8, device=device)
+        self.m_scale = torch.zeros(self.gtotal, dtype=torch.int16, device=device)
+        if adam:
+            self.v_q = torch.zeros(self.total, dtype=torch.uint8, device=device)
+            self.v_scale = torch.zeros(self.gtotal, dtype=torch.int16, device=device)
+        else:
+            self.v_q = self.v_scale = None
+        self.states = [self._state(i) for i in range(len(self.numels))]
+
+    def _state(self, i: int) -> fo.TensorState:
+        o, g, n = self.offsets[i], self.goffsets[i], self.numels[i]
+        ng = (n + 31) // 32
+        sl = lambda t, a, k: None if t is None else t[a:a + k]
+        return fo.TensorState(self.w[o:o + n], self.ecc[o:o + n], self.m_q[o:o + n],
+                              self.m_scale[g:g + ng], sl(self.v_q, o, n), sl(self.v_scale, g, ng))
+
+    @property
+    def format_bits(self) -> int:
+        return self.ecc_bits
+
+    def nbytes(self) -> int:
+        t = self.w.nbytes + self.ecc.nbytes + self.m_q.nbytes + self.m_scale.nbytes
+        if self.adam:
+            t += self.v_q.nbytes + self.v_scale.nbytes
+        return t
+
+    def encode_from(self, i: int, x32, stream=None):
+        """Split f32 masters of tensor i into downcast + ECC (device kernel)."""
+        st = self.states[i]
+        fmt = fo.make_format(self.w_dtype, "bf16", self.ecc_bits)
+        fo.fo_encode_master(x32, st.w, st.ecc, st.numel, fmt, stream)
+
+    def decode_to(self, i: int, out32, stream=None):
+        st = self.states[i]
+        fmt = fo.make_format(self.w_dtype, "bf16", self.ecc_bits)
+        fo.fo_decode_master(st.w, st.ecc, out32, st.numel, fmt, stream)
+
+
+class CompressedAdamW:
+    """AdamW over a parameter list with bf16/fp16 + ECC masters and 8-bit
+    companded states; ``step`` is one fused kernel launch for the whole list
+    (or one per call when used for gradient release)."""
+
+    def __init__(self, params: CompressedParams, lr=1e-3, betas=(0.9, 0.999), eps=1e-8,
+                 weight_decay=0.01, grad_dtype="bf16"):
+        assert params.adam
+        self.p = params
+        self.hp = dict(lr=lr, beta1=betas[0], beta2=betas[1], eps=eps, weight_decay=weight_decay)
+        self.t = 0
+        self.fmt = fo.make_format(params.w_dtype, grad_dtype, params.ecc_bits)
+
+    def hparams(self, t: int) -> fo.fo_adamw_hparams:
+        h = self.hp
+        return fo.fo_adamw_hparams(h["lr"], h["beta1"], h["beta2"], h["eps"], h["weight_decay"], t)
+
+    def step(self, grads, stream=None):
+        self.t += 1
+        descs = fo.descriptors(self.p.states, grads)
+        fo.fo_adamw_step(descs, len(self.p.states), self.fmt, self.hparams(self.t), stream)
+
+    def step_tensor(self, i: int, grad, t: int, stream=None):
+        """Gradient release: step tensor i alone (its gradient may be freed
+        once the work on the stream has finished)."""
+        descs = fo.descriptors([self.p.states[i]], [grad])
+        fo.fo_adamw_step(descs, 1, self.fmt, self.hparams(t), stream)
+
+
+class CompressedSGDM:
+    def __init__(self, params: CompressedParams, lr=0.1, momentum=0.9, dampening=0.0,
+                 weight_decay=0.0, nesterov=False, grad_dtype="fp16"):
+        self.p = params
+        self.hp = dict(lr=lr, momentum=momentum, dampening=dampening, weight_decay=weight_decay,
+                       nesterov=int(bool(nesterov)))
+        self.t = 0
+        self.fmt = fo.make_format(params.w_dtype, grad_dtype, params.ecc_bits)
+
+    def hparams(self, t: int) -> fo.fo_sgdm_hparams:
+        h = self.hp
+        return fo.fo_sgdm_hparams(h["lr"], h["momentum"], h["dampening"], h["weight_decay"],
+                                  h["nesterov"], t)
+
+    def step(self, grads, stream=None):
+        self.t += 1
+        descs = fo.descriptors(self.p.states, grads)
+        fo.fo_sgdm_step(descs, len(self.p.states), self.fmt, self.hparams(self.t), stream)

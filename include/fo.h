@@ -60,6 +60,12 @@
 
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define FO_API __attribute__((visibility("default")))
+#else
+#define FO_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -129,7 +135,7 @@ typedef struct {
  * not finite, beta outside [0, 1)), FO_ERR_UNSUPPORTED, FO_ERR_ALIGNMENT,
  * FO_ERR_TOO_MANY_TENSORS, FO_ERR_CUDA.
  */
-fo_status fo_adamw_step(const fo_tensor* t, int n_tensors, fo_format f,
+FO_API fo_status fo_adamw_step(const fo_tensor* t, int n_tensors, fo_format f,
                         const fo_adamw_hparams* h, void* stream);
 
 /*
@@ -138,7 +144,7 @@ fo_status fo_adamw_step(const fo_tensor* t, int n_tensors, fo_format f,
  * support and error behaviour as fo_adamw_step; momentum and dampening must
  * lie in [0, 1].
  */
-fo_status fo_sgdm_step(const fo_tensor* t, int n_tensors, fo_format f,
+FO_API fo_status fo_sgdm_step(const fo_tensor* t, int n_tensors, fo_format f,
                        const fo_sgdm_hparams* h, void* stream);
 
 /*
@@ -149,7 +155,7 @@ fo_status fo_sgdm_step(const fo_tensor* t, int n_tensors, fo_format f,
  * FO_ERR_UNSUPPORTED, FO_ERR_ALIGNMENT (x32 not 4-byte aligned, w or int16
  * ecc not 2-byte aligned), FO_ERR_CUDA.
  */
-fo_status fo_encode_master(const float* x32, void* w, void* ecc, int64_t n, fo_format f,
+FO_API fo_status fo_encode_master(const float* x32, void* w, void* ecc, int64_t n, fo_format f,
                            void* stream);
 
 /*
@@ -157,18 +163,18 @@ fo_status fo_encode_master(const float* x32, void* w, void* ecc, int64_t n, fo_f
  * ecc (device).  Used to export checkpoints.  Same errors as
  * fo_encode_master.  Non-finite x' decode to x' itself.
  */
-fo_status fo_decode_master(const void* w, const void* ecc, float* x32, int64_t n, fo_format f,
+FO_API fo_status fo_decode_master(const void* w, const void* ecc, float* x32, int64_t n, fo_format f,
                            void* stream);
 
 /* Static English name of a status code. */
-const char* fo_status_string(fo_status s);
+FO_API const char* fo_status_string(fo_status s);
 
 /* Detail of the last non-FO_OK status returned on the calling thread
    ("" if none).  The pointer stays valid until the next call on the thread. */
-const char* fo_last_error(void);
+FO_API const char* fo_last_error(void);
 
 /* Library version as major * 10000 + minor * 100 + patch. */
-int fo_version(void);
+FO_API int fo_version(void);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,315 @@
+"""GPU parity: every byte the CUDA path emits (downcast weights, ECC codes,
+momentum / variance codes, fp16 scales) equals the CPU oracle's, on the same
+seeded inputs.  All GPU work goes through the C ABI (libfo.so via ctypes).
+
+Bar: bit-exact on every emitted byte (the method emits integer codes and
+16-bit patterns only).  Non-finite values are not produced by these inputs.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_states_b200 import fo
+from bit_states_b200.state import CompressedParams
+from workloads import gen, workload
+from workloads import device as wdev
+from workloads.shapes import TensorSpec, Workload, ADAMW_HP, SGDM_HP
+
+import gpu_util as U
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    from bit_states_b200 import build as fobuild
+
+    fobuild.build()
+    wdev.build()
+    fo.load()
+    torch.cuda.init()
+    yield
+    torch.cuda.synchronize()
+
+
+def _nthreads():
+    import os
+
+    return max(1, min(32, os.cpu_count() or 1))
+
+
+# ---- generator -----------------------------------------------------------------
+
+@pytest.mark.parametrize("name", ["gpt2-small-124M", "resnet50-25.6M", "llama3.1-8b"])
+def test_device_generator_matches_host(name):
+    wl = workload(name)
+    rng = np.random.default_rng(0)
+    for ti in rng.choice(len(wl.tensors), size=min(6, len(wl.tensors)), replace=False):
+        n = wl.tensors[ti].numel
+        n_dev = min(n, 1 << 22)
+        x = torch.empty(n_dev, dtype=torch.float32, device=DEV)
+        g = torch.empty(n_dev, dtype=torch.int16, device=DEV)
+        # device generation is by global index, so generate a prefix
+        spec = wl.tensors[ti]
+        if spec.init != "const":
+            wdev.master_f32(wl, ti, x)
+        wdev.grad_16(wl, ti, 3, g)
+        idx = rng.choice(n_dev, size=min(n_dev, 20000), replace=False)
+        if spec.init != "const":
+            assert np.array_equal(x.cpu().numpy()[idx].view(np.uint32),
+                                  wl.master_values(ti, idx).view(np.uint32))
+        assert np.array_equal(g.cpu().numpy()[idx].view(np.uint16), wl.grad_bits(ti, 3, idx))
+
+
+# ---- master codec ---------------------------------------------------------------
+
+def _codec_inputs(wdt):
+    rng = np.random.default_rng(7)
+    if wdt == "bf16":
+        heads = np.arange(1 << 16, dtype=np.int64)
+        heads = heads[(heads & 0x7F80) != 0x7F80]
+        offs = np.unique(np.concatenate([256 * np.arange(-128, 128)[:, None] + 128 + np.array([-1, 0, 1])[None, :]]
+                                        ).ravel().tolist() + [0, 1, -1, 32767, -32767, -32768])
+        m = ((heads & 0x7FFF) << 16)[:, None] + offs[None, :]
+        ok = (m >= 0) & (m < 0x7F800000)
+        pats = (((heads & 0x8000) << 16)[:, None] | m)[ok].astype(np.uint32)
+    else:
+        e = np.arange(256, dtype=np.uint32) << 23
+        tails = np.concatenate([np.arange(0, 1 << 13, dtype=np.uint32), rng.integers(0, 1 << 23, 4096).astype(np.uint32)])
+        pats = (e[:, None] | tails[None, :]).ravel()
+        pats = np.concatenate([pats, pats | np.uint32(0x80000000)])
+    r = rng.integers(0, 1 << 32, size=1 << 22, dtype=np.uint64).astype(np.uint32)
+    pats = np.concatenate([pats, r])
+    x = pats.view(np.float32)
+    return x[np.isfinite(x)]
+
+
+@pytest.mark.parametrize("wdt", ["bf16", "fp16"])
+@pytest.mark.parametrize("nbits", [8, 16])
+def test_encode_decode_master_bit_exact(wdt, nbits):
+    x = _codec_inputs(wdt)
+    n = x.size
+    fmt = fo.make_format(wdt, "bf16", nbits)
+    xd = torch.from_numpy(x).to(DEV)
+    w = torch.empty(n, dtype=torch.int16, device=DEV)
+    e = torch.empty(n, dtype=torch.int8 if nbits == 8 else torch.int16, device=DEV)
+    fo.fo_encode_master(xd, w, e, n, fmt)
+    ow, oe = oracle.encode_master(x, U.DT[wdt], nbits, threads=_nthreads())
+    gw = w.cpu().numpy().view(np.uint16)
+    ge = e.cpu().numpy()
+    assert np.count_nonzero(gw != ow) == 0
+    assert np.count_nonzero(ge != oe) == 0
+    # decode of every code of random heads (not just encode outputs)
+    rng = np.random.default_rng(11)
+    heads = rng.integers(0, 1 << 16, size=1 << 20, dtype=np.uint32).astype(np.uint16)
+    lim = (1 << (nbits - 1)) - 1
+    codes = rng.integers(-lim, lim + 1, size=heads.size).astype(oracle.ecc_dtype(nbits))
+    od = oracle.decode_master(heads, codes, U.DT[wdt], nbits, threads=_nthreads())
+    xo = torch.empty(heads.size, dtype=torch.float32, device=DEV)
+    fo.fo_decode_master(torch.from_numpy(heads.view(np.int16)).to(DEV), torch.from_numpy(codes).to(DEV),
+                        xo, heads.size, fmt)
+    gd = xo.cpu().numpy()
+    nan = np.isnan(od)
+    assert np.array_equal(np.isnan(gd), nan)
+    assert np.count_nonzero(gd.view(np.uint32)[~nan] != od.view(np.uint32)[~nan]) == 0
+
+
+# ---- flat group, 10 steps, every byte ----------------------------------------------
+
+def _run_full_compare(wl, steps, order=None, check_every=True):
+    P = U.device_state(wl)
+    G = U.GradArena(P)
+    orcs = []
+    for ti, t in enumerate(wl.tensors):
+        orcs.append(U.OracleSample(wl, ti, np.arange((t.numel + 31) // 32), threads=_nthreads()))
+    for t in range(1, steps + 1):
+        G.fill(wl, t)
+        U.step(wl, P, G, t, order=order)
+        for o in orcs:
+            o.step(t)
+        if check_every or t == steps:
+            torch.cuda.synchronize()
+            for ti, o in enumerate(orcs):
+                exp = o.expected()
+                got = U.gather_device(P, ti, exp)
+                mm = U.mismatches(exp, got)
+                assert all(v == 0 for v in mm.values()), (wl.name, ti, t, mm)
+    return P
+
+
+def test_flat_1m_ten_adamw_steps_every_byte():
+    wl = workload("flat-1M")
+    _run_full_compare(wl, 10)
+
+
+# ---- ragged sizes, misaligned views, all formats ------------------------------------
+
+RAGGED = [1, 2, 31, 32, 33, 255, 256, 257, 511, 512, 513, 1000, 4095, 4096, 65537]
+
+
+def _ragged_workload(opt, wdt, gdt, nbits):
+    ts = [TensorSpec(f"t{i}", (n,), "normal", 0.02 if i % 3 else 1.5) for i, n in enumerate(RAGGED)]
+    hp = dict(ADAMW_HP) if opt == "adamw" else dict(SGDM_HP)
+    return Workload(name=f"ragged-{opt}", tensors=ts, optimizer=opt, hparams=hp, w_dtype=wdt,
+                    grad_dtype=gdt, ecc_bits=nbits, grad_dist="normal_outliers", grad_scale=1e-3, seed=5)
+
+
+@pytest.mark.parametrize("opt", ["adamw", "sgdm"])
+@pytest.mark.parametrize("wdt,gdt", [("bf16", "bf16"), ("fp16", "fp16"), ("bf16", "fp16"), ("fp16", "bf16")])
+@pytest.mark.parametrize("nbits", [8, 16])
+def test_ragged_multitensor_all_formats(opt, wdt, gdt, nbits):
+    wl = _ragged_workload(opt, wdt, gdt, nbits)
+    _run_full_compare(wl, 3)
+
+
+@pytest.mark.parametrize("nesterov,damp", [(1, 0.0), (0, 0.25)])
+def test_sgdm_variants(nesterov, damp):
+    wl = _ragged_workload("sgdm", "fp16", "fp16", 8)
+    wl.hparams.update(nesterov=nesterov, dampening=damp)
+    _run_full_compare(wl, 3)
+
+
+@pytest.mark.parametrize("shift", [1, 2, 3, 8, 16])
+def test_misaligned_views_take_scalar_path(shift):
+    """Tensors whose arrays start off the 32-byte grid (views into a larger
+    buffer) give the same bytes; canaries around every output stay intact."""
+    n = 3000
+    wl = _ragged_workload("adamw", "bf16", "bf16", 8)
+    wl.tensors = [TensorSpec("a", (n,), "normal", 0.02)]
+    idx = np.arange(n)
+    x = wl.master_values(0, idx)
+    ow, oe = oracle.encode_master(x, 0, 8)
+    pad = 64
+    mk = lambda dt, cnt: torch.full((cnt + 2 * pad,), 0x5A, dtype=dt, device=DEV)
+    w = mk(torch.int16, n); e = mk(torch.int8, n); mq = mk(torch.int8, n); vq = mk(torch.uint8, n)
+    ng = (n + 31) // 32
+    ms = mk(torch.int16, ng); vs = mk(torch.int16, ng); g = mk(torch.int16, n)
+    s = shift
+    wv, ev, mqv, vqv, gv = w[pad + s:pad + s + n], e[pad + s:pad + s + n], mq[pad + s:pad + s + n], \
+        vq[pad + s:pad + s + n], g[pad + s:pad + s + n]
+    msv, vsv = ms[pad + 1:pad + 1 + ng], vs[pad + 1:pad + 1 + ng]
+    wv.copy_(torch.from_numpy(ow.view(np.int16))); ev.copy_(torch.from_numpy(oe))
+    mqv.zero_(); vqv.zero_(); msv.zero_(); vsv.zero_()
+    st = oracle.State.zeros_like_master(ow, oe)
+    before = {k: v.clone() for k, v in dict(w=w, e=e, mq=mq, vq=vq, ms=ms, vs=vs).items()}
+    state = fo.TensorState(wv, ev, mqv, msv, vqv, vsv)
+    for t in (1, 2):
+        gb = wl.grad_bits(0, t, idx)
+        gv.copy_(torch.from_numpy(gb.view(np.int16)))
+        d = fo.descriptors([state], [gv])
+        fo.fo_adamw_step(d, 1, fo.make_format(), U.hparams_adamw(wl, t))
+        oracle.adamw_step(st, gb, **wl.hparams, step=t)
+    torch.cuda.synchronize()
+    assert np.array_equal(U.to_np_bytes(wv), st.w)
+    assert np.array_equal(ev.cpu().numpy(), st.ecc)
+    assert np.array_equal(mqv.cpu().numpy(), st.mq)
+    assert np.array_equal(vqv.cpu().numpy(), st.vq)
+    assert np.array_equal(U.to_np_bytes(msv), st.ms)
+    assert np.array_equal(U.to_np_bytes(vsv), st.vs)
+    for k, full in dict(w=w, e=e, mq=mq, vq=vq, ms=ms, vs=vs).items():
+        lo = pad + (1 if k in ("ms", "vs") else s)
+        cnt = ng if k in ("ms", "vs") else n
+        assert torch.equal(full[:lo], before[k][:lo]), k
+        assert torch.equal(full[lo + cnt:], before[k][lo + cnt:]), k
+
+
+def test_empty_and_tiny_tensors_in_one_call():
+    wl = _ragged_workload("adamw", "bf16", "bf16", 8)
+    wl.tensors = [TensorSpec("one", (1,), "normal", 0.02), TensorSpec("seven", (7,), "normal", 0.02)]
+    P = U.device_state(wl)
+    G = U.GradArena(P)
+    G.fill(wl, 1)
+    empty = fo.TensorState(P.w[:0], P.ecc[:0], P.m_q[:0], P.m_scale[:0], P.v_q[:0], P.v_scale[:0])
+    states = [empty, P.states[0], empty, P.states[1]]
+    grads = [G.buf[:0], G.views[0], G.buf[:0], G.views[1]]
+    d = fo.descriptors(states, grads)
+    fo.fo_adamw_step(d, 4, fo.make_format(), U.hparams_adamw(wl, 1))
+    torch.cuda.synchronize()
+    for ti in range(2):
+        o = U.OracleSample(wl, ti, np.arange(1))
+        o.step(1)
+        exp = o.expected()
+        assert all(v == 0 for v in U.mismatches(exp, U.gather_device(P, ti, exp)).values())
+
+
+# ---- gradient release == one multi-tensor launch -------------------------------------
+
+def test_release_order_equals_multitensor_gpt2_shapes():
+    wl = workload("gpt2-small-124M")
+    A = U.device_state(wl)
+    B = U.device_state(wl)
+    G = U.GradArena(A)
+    order = list(range(len(wl.tensors)))[::-1]
+    for t in (1, 2, 3):
+        G.fill(wl, t)
+        U.step(wl, A, G, t)
+        U.step(wl, B, G, t, order=order)
+    torch.cuda.synchronize()
+    for name in ("w", "ecc", "m_q", "m_scale", "v_q", "v_scale"):
+        assert torch.equal(getattr(A, name), getattr(B, name)), name
+
+
+# ---- full-size workloads in the benchmark's launch configuration ---------------------
+
+def _sampled_check(wl, P, orcs, tag):
+    torch.cuda.synchronize()
+    bad = {}
+    for ti, o in orcs.items():
+        exp = o.expected()
+        mm = U.mismatches(exp, U.gather_device(P, ti, exp))
+        if any(mm.values()):
+            bad[ti] = mm
+    assert not bad, (wl.name, tag, bad)
+
+
+def test_gpt2_small_101_steps_sampled():
+    """GPT-2-small parameter list, 100 warm steps + 1 (the benchmark's
+    workload of this size), one multi-tensor launch per step; the oracle
+    replays the same seeded inputs for 2 sampled groups per tensor (plus the
+    first and last group) over all 101 steps; bytes compared at 1, 100, 101."""
+    wl = workload("gpt2-small-124M")
+    P = U.device_state(wl)
+    G = U.GradArena(P)
+    rng = np.random.default_rng(1)
+    orcs = {ti: U.OracleSample(wl, ti, U.sample_groups(t.numel, 2, rng)) for ti, t in enumerate(wl.tensors)}
+    for t in range(1, wl.warm_steps + 2):
+        G.fill(wl, t)
+        U.step(wl, P, G, t)
+        for o in orcs.values():
+            o.step(t)
+        if t in (1, 100, 101):
+            _sampled_check(wl, P, orcs, f"step {t}")
+
+
+def test_resnet50_sgdm_every_byte():
+    wl = workload("resnet50-25.6M")
+    _run_full_compare(wl, 2)
+
+
+@pytest.mark.parametrize("mode", ["multi", "release", "ecc16"])
+def test_llama_8b_sampled(mode):
+    """Llama-3.1-8B parameter list at full size (8.03e9 parameters): one
+    multi-tensor launch (the benchmark's configuration), the 291 per-tensor
+    calls in reverse layer order, and the 16-bit-ECC variant; sampled groups
+    of every tensor against the oracle."""
+    if mode == "ecc16":
+        wl = workload("llama3.1-8b-ecc16")
+    else:
+        wl = workload("llama3.1-8b")
+    P = U.device_state(wl)
+    G = U.GradArena(P)
+    G.fill(wl, 1)
+    order = list(range(len(wl.tensors)))[::-1] if mode == "release" else None
+    U.step(wl, P, G, 1, order=order)
+    rng = np.random.default_rng(2)
+    orcs = {ti: U.OracleSample(wl, ti, U.sample_groups(t.numel, 48, rng)) for ti, t in enumerate(wl.tensors)}
+    for o in orcs.values():
+        o.step(1)
+    _sampled_check(wl, P, orcs, mode)
+    del P, G
+    torch.cuda.empty_cache()
