@@ -87,7 +87,9 @@ def sample_groups(n, k, rng):
 
 
 def group_elems(n, groups):
-    return np.concatenate([np.arange(32 * g, min(32 * g + 32, n)) for g in groups]).astype(np.int64)
+    g = np.asarray(groups, np.int64)
+    idx = (32 * g[:, None] + np.arange(32, dtype=np.int64)[None, :]).ravel()
+    return idx[idx < n]
 
 
 class OracleSample:

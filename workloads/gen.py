@@ -53,6 +53,7 @@ def _mix_int(z: int) -> int:
 
 
 def stream_key(seed: int, tensor: int, step: int, kind: int) -> int:
+    seed, tensor, step, kind = int(seed), int(tensor), int(step), int(kind)
     k = _mix_int((seed + 1) * GAMMA)
     k = _mix_int(k ^ (((tensor + 1) * GAMMA) & MASK))
     k = _mix_int(k ^ (((step + 1) * GAMMA) & MASK))
