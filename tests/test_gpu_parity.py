@@ -313,3 +313,82 @@ def test_llama_8b_sampled(mode):
     _sampled_check(wl, P, orcs, mode)
     del P, G
     torch.cuda.empty_cache()
+
+
+# ---- exact rounding ties of the 8-bit codes ------------------------------------------
+
+def _tie_groups(n_groups=96, seed=3):
+    """bf16 gradients whose step-1 momentum / variance codes land exactly on
+    a half-integer before rounding (127*c or sqrt(v)*k == q + 0.5), so that a
+    code computed with one rounding fewer (a fused multiply-add) would differ.
+    Found by a binary32 numpy search; element 0 of a group fixes its scale."""
+    f = np.float32
+    rng = np.random.default_rng(seed)
+    allg = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    gv = (allg.astype(np.uint32) << 16).view(np.float32)
+    ok = np.isfinite(gv) & (np.abs(gv) > 1e-12)
+    groups = []
+    for _ in range(n_groups * 400):
+        G = f(rng.uniform(2e-4, 5e-3))
+        Gb = gen.to_16bit(np.array([G], np.float32), "bf16")[0]
+        G = np.array([Gb], np.uint16).astype(np.uint32) << 16
+        G = G.view(np.float32)[0]
+        cand = ok & (np.abs(gv) < abs(G))
+        g = gv[cand]
+        mn = (f(0.1) * g).astype(np.float32)
+        A = abs(f(f(0.1) * G))
+        S = oracle.scale_fp16(np.array([A], np.float32))[0]
+        Sf = np.array([S], np.uint16).view(np.float16).astype(np.float32)[0]
+        r = f(1) / Sf
+        y = (mn * r).astype(np.float32)
+        c = ((f(2) * y) / (f(1) + np.abs(y))).astype(np.float32)
+        t = (f(127) * c).astype(np.float32)
+        tie_m = (t - np.floor(t)) == f(0.5)
+        vn = (f(1 - 0.999) * (g * g)).astype(np.float32)
+        s = np.sqrt(vn)
+        Av = np.sqrt(f(f(1 - 0.999) * (G * G)))
+        Sv = oracle.scale_fp16(np.array([Av], np.float32))[0]
+        Svf = np.array([Sv], np.uint16).view(np.float16).astype(np.float32)[0]
+        tv = (s * (f(255) / Svf)).astype(np.float32)
+        tie_v = (tv - np.floor(tv)) == f(0.5)
+        pick = np.nonzero(tie_m | tie_v)[0]
+        if pick.size < 1:
+            continue
+        sel = rng.choice(pick, size=min(31, pick.size), replace=False)
+        fill = rng.choice(g.size, size=31 - sel.size, replace=False)
+        grp = np.concatenate([[G], g[sel], g[fill]]).astype(np.float32)
+        groups.append(grp)
+        if len(groups) == n_groups:
+            break
+    assert len(groups) >= 16
+    return np.concatenate(groups)
+
+
+@pytest.mark.parametrize("shift", [0, 1])
+def test_code_rounding_ties_bit_exact(shift):
+    g32 = _tie_groups()
+    n = g32.size
+    gb = gen.to_16bit(g32, "bf16")
+    rng = np.random.default_rng(9)
+    x = (rng.standard_normal(n) * 0.02).astype(np.float32)
+    w, e = oracle.encode_master(x, 0, 8)
+    st = oracle.State.zeros_like_master(w, e)
+    pad = 64
+    ng = (n + 31) // 32
+    bufs = [torch.zeros(n + pad, dtype=dt, device=DEV) for dt in (torch.int16, torch.int8, torch.int8, torch.uint8, torch.int16)]
+    sc = [torch.zeros(ng + pad, dtype=torch.int16, device=DEV) for _ in range(2)]
+    wv, ev, mqv, vqv, gv = (b[shift:shift + n] for b in bufs)
+    wv.copy_(torch.from_numpy(w.view(np.int16)))
+    ev.copy_(torch.from_numpy(e))
+    gv.copy_(torch.from_numpy(gb.view(np.int16)))
+    dst = fo.TensorState(wv, ev, mqv, sc[0][:ng], vqv, sc[1][:ng])
+    hp = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01)
+    fo.fo_adamw_step(fo.descriptors([dst], [gv]), 1, fo.make_format(), fo.fo_adamw_hparams(**hp, step=1))
+    oracle.adamw_step(st, gb, **hp, step=1)
+    torch.cuda.synchronize()
+    assert np.array_equal(mqv.cpu().numpy(), st.mq)
+    assert np.array_equal(vqv.cpu().numpy(), st.vq)
+    assert np.array_equal(U.to_np_bytes(sc[0][:ng]), st.ms)
+    assert np.array_equal(U.to_np_bytes(sc[1][:ng]), st.vs)
+    assert np.array_equal(U.to_np_bytes(wv), st.w)
+    assert np.array_equal(ev.cpu().numpy(), st.ecc)
