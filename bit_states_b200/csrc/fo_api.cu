@@ -101,30 +101,44 @@ StepKernel pick_step(const fo_format& f)
     return nullptr;
 }
 
-struct OccCache {
+struct LaunchCache {
     std::mutex mu;
-    const void* fn[64] = {};
-    int blocks[64] = {};
+    int dev[128] = {};
+    const void* fn[128] = {};
+    int blocks[128] = {};
     int n = 0;
-} g_occ;
+} g_launch;
 
-int blocks_per_sm(StepKernel k)
+// once per (device, kernel): allow the dynamic shared memory of the stage
+// buffers and find how many blocks fit on one SM
+fo_status prepare_kernel(StepKernel k, int smem, int* blocks_per_sm)
 {
-    std::lock_guard<std::mutex> lock(g_occ.mu);
-    for (int i = 0; i < g_occ.n; i++)
-        if (g_occ.fn[i] == (const void*)k) return g_occ.blocks[i];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    std::lock_guard<std::mutex> lock(g_launch.mu);
+    for (int i = 0; i < g_launch.n; i++)
+        if (g_launch.fn[i] == (const void*)k && g_launch.dev[i] == dev) {
+            *blocks_per_sm = g_launch.blocks[i];
+            return FO_OK;
+        }
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
     int b = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, k, fo::kThreads, 0) != cudaSuccess || b < 1)
-        b = 1;
-    if (g_occ.n < 64) {
-        g_occ.fn[g_occ.n] = (const void*)k;
-        g_occ.blocks[g_occ.n] = b;
-        g_occ.n++;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, k, fo::kThreads, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    if (b < 1) b = 1;
+    if (g_launch.n < 128) {
+        g_launch.fn[g_launch.n] = (const void*)k;
+        g_launch.dev[g_launch.n] = dev;
+        g_launch.blocks[g_launch.n] = b;
+        g_launch.n++;
     }
-    return b;
+    *blocks_per_sm = b;
+    return FO_OK;
 }
 
-fo_status launch_step(StepKernel k, const fo::Scalars& sc, const fo_tensor* t, int n,
+fo_status launch_step(StepKernel k, int smem, const fo::Scalars& sc, const fo_tensor* t, int n,
                       cudaStream_t stream)
 {
     bool any = false;
@@ -133,7 +147,9 @@ fo_status launch_step(StepKernel k, const fo::Scalars& sc, const fo_tensor* t, i
     int sms = 0;
     fo_status st = device_sms(&sms);
     if (st != FO_OK) return st;
-    const int bps = blocks_per_sm(k);
+    int bps = 1;
+    st = prepare_kernel(k, smem, &bps);
+    if (st != FO_OK) return st;
     // kernel parameters are copied at launch, so one block of host memory
     // per thread serves every launch
     thread_local fo::StepParams P;
@@ -156,6 +172,10 @@ fo_status launch_step(StepKernel k, const fo::Scalars& sc, const fo_tensor* t, i
             d.vq = x.v_q;
             d.vs = x.v_scale;
             d.numel = x.numel;
+            const uintptr_t a = (uintptr_t)x.w | (uintptr_t)x.grad | (uintptr_t)x.ecc | (uintptr_t)x.m_q |
+                                (uintptr_t)x.m_scale | (uintptr_t)x.v_q | (uintptr_t)x.v_scale;
+            d.aligned16 = (a & 15u) == 0 ? 1 : 0;
+            d.reserved = 0;
             chunks += (x.numel + fo::kChunk - 1) / fo::kChunk;
             P.chunk_start[++m] = chunks;
         }
@@ -164,11 +184,10 @@ fo_status launch_step(StepKernel k, const fo::Scalars& sc, const fo_tensor* t, i
         P.total_chunks = chunks;
         // a sentinel past the last tensor keeps the device-side walk bounded
         for (int j = m + 1; j <= fo::kMaxTensorsPerLaunch; j++) P.chunk_start[j] = INT64_MAX;
-        const int64_t warps_per_block = fo::kThreads / 32;
-        int64_t grid = (chunks + warps_per_block - 1) / warps_per_block;
+        int64_t grid = (chunks + fo::kWarps - 1) / fo::kWarps;
         const int64_t cap = (int64_t)sms * bps;
         if (grid > cap) grid = cap;
-        k<<<(unsigned)grid, fo::kThreads, 0, stream>>>(P);
+        k<<<(unsigned)grid, fo::kThreads, smem, stream>>>(P);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "step kernel launch");
     }
@@ -176,6 +195,11 @@ fo_status launch_step(StepKernel k, const fo::Scalars& sc, const fo_tensor* t, i
 }
 
 bool is_finite(double v) { return std::isfinite(v); }
+
+int stage_smem(const fo_format& f)
+{
+    return f.ecc_bits == 8 ? fo::step_smem_bytes<8>() : fo::step_smem_bytes<16>();
+}
 
 int64_t grid_for(int64_t n, int sms)
 {
@@ -218,7 +242,7 @@ fo_status fo_adamw_step(const fo_tensor* t, int n_tensors, fo_format f, const fo
     sc.s[7] = (float)(1.0 - h->lr * h->weight_decay);
     StepKernel k = pick_step<fo::kAdamW>(f);
     if (!k) return fail(FO_ERR_UNSUPPORTED, "format not provided");
-    return launch_step(k, sc, t, n_tensors, (cudaStream_t)stream);
+    return launch_step(k, stage_smem(f), sc, t, n_tensors, (cudaStream_t)stream);
 }
 
 fo_status fo_sgdm_step(const fo_tensor* t, int n_tensors, fo_format f, const fo_sgdm_hparams* h,
@@ -247,7 +271,7 @@ fo_status fo_sgdm_step(const fo_tensor* t, int n_tensors, fo_format f, const fo_
     sc.s[7] = 0.0f;
     StepKernel k = pick_step<fo::kSGDM>(f);
     if (!k) return fail(FO_ERR_UNSUPPORTED, "format not provided");
-    return launch_step(k, sc, t, n_tensors, (cudaStream_t)stream);
+    return launch_step(k, stage_smem(f), sc, t, n_tensors, (cudaStream_t)stream);
 }
 
 fo_status fo_encode_master(const float* x32, void* w, void* ecc, int64_t n, fo_format f, void* stream)
