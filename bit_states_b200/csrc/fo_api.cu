@@ -138,7 +138,7 @@ fo_status prepare_kernel(StepKernel k, int smem, int* blocks_per_sm)
     return FO_OK;
 }
 
-fo_status launch_step(StepKernel k, int smem, const fo::Scalars& sc, int fast_math, const fo_tensor* t, int n,
+fo_status launch_step(StepKernel k, int smem, const fo::Scalars& sc, const fo_tensor* t, int n,
                       cudaStream_t stream)
 {
     bool any = false;
@@ -157,7 +157,6 @@ fo_status launch_step(StepKernel k, int smem, const fo::Scalars& sc, int fast_ma
     while (i < n) {
         std::memset(&P, 0, offsetof(fo::StepParams, t));
         P.sc = sc;
-        P.fast_math = fast_math;
         int m = 0;
         int64_t chunks = 0;
         P.chunk_start[0] = 0;
@@ -241,17 +240,9 @@ fo_status fo_adamw_step(const fo_tensor* t, int n_tensors, fo_format f, const fo
     sc.s[5] = (float)(1.0 / std::sqrt(bc2));
     sc.s[6] = (float)h->eps;
     sc.s[7] = (float)(1.0 - h->lr * h->weight_decay);
-    // The kernel's Newton-Raphson square root and division are exact within
-    // ranges that these hyper-parameters guarantee (betas 0 or in
-    // [0.5, 1 - 2^-10] resp. [0.5, 1 - 2^-14], eps in [2^-60, 1]); otherwise it
-    // uses the IEEE operations.
-    const double b1 = h->beta1, b2 = h->beta2;
-    const int fast_math = (b1 == 0.0 || (b1 >= 0.5 && 1.0 - b1 >= 0x1p-10)) &&
-                          (b2 == 0.0 || (b2 >= 0.5 && 1.0 - b2 >= 0x1p-14)) &&
-                          h->eps >= 0x1p-60 && h->eps <= 1.0;
     StepKernel k = pick_step<fo::kAdamW>(f);
     if (!k) return fail(FO_ERR_UNSUPPORTED, "format not provided");
-    return launch_step(k, stage_smem(f), sc, fast_math, t, n_tensors, (cudaStream_t)stream);
+    return launch_step(k, stage_smem(f), sc, t, n_tensors, (cudaStream_t)stream);
 }
 
 fo_status fo_sgdm_step(const fo_tensor* t, int n_tensors, fo_format f, const fo_sgdm_hparams* h,
@@ -280,7 +271,7 @@ fo_status fo_sgdm_step(const fo_tensor* t, int n_tensors, fo_format f, const fo_
     sc.s[7] = 0.0f;
     StepKernel k = pick_step<fo::kSGDM>(f);
     if (!k) return fail(FO_ERR_UNSUPPORTED, "format not provided");
-    return launch_step(k, stage_smem(f), sc, 0, t, n_tensors, (cudaStream_t)stream);
+    return launch_step(k, stage_smem(f), sc, t, n_tensors, (cudaStream_t)stream);
 }
 
 fo_status fo_encode_master(const float* x32, void* w, void* ecc, int64_t n, fo_format f, void* stream)
