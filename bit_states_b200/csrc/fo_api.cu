@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <limits>
 #include <mutex>
 #include <string>
 
@@ -213,6 +214,34 @@ int64_t grid_for(int64_t n, int sms)
 
 extern "C" {
 
+// Bounds of the kernel's fast path for AdamW (its Newton-Raphson update; see
+// lane_adamw_fast): s[8] = -lr/(1-b1^t) * 2^-40, s[9] = the smallest
+// |x (1-lr wd)| for which an update of at most
+//   U = |lr/(1-b1^t)| (2^-119 / eps + 2^-126)
+// cannot change x'' (U < |x (1-lr wd)| 2^-26), s[10] = the largest sqrt(v')
+// that keeps the divisor sqrt(v') / sqrt(1-b2^t) + eps at or below 2^20.
+// Where those conditions cannot hold (eps < 2^-60, a step size too small to
+// scale by 2^-40) s[9] is +inf and every slice takes the exact path.
+static void adamw_fast_bounds(fo::Scalars& sc)
+{
+    const float step = sc.s[4], ibc2 = sc.s[5], eps = sc.s[6];
+    const float inf = std::numeric_limits<float>::infinity();
+    sc.s[8] = -step * 0x1p-40f;
+    const bool ok = eps >= 0x1p-60f && eps < 0x1p19f && (step == 0.0f || std::fabs(step) >= 0x1p-80f);
+    if (!ok) {
+        sc.s[9] = inf;
+        sc.s[10] = 0.0f;
+        return;
+    }
+    const double u = std::fabs((double)step) * (std::ldexp(1.0, -119) / (double)eps + std::ldexp(1.0, -126));
+    const double thr = u * std::ldexp(1.0, 26) * (1.0 + std::ldexp(1.0, -10));
+    float t = (float)thr;
+    if ((double)t < thr) t = std::nextafter(t, inf);
+    sc.s[9] = t;
+    float b = (float)((std::ldexp(1.0, 20) - (double)eps) / (double)ibc2 * (1.0 - std::ldexp(1.0, -20)));
+    sc.s[10] = b;
+}
+
 fo_status fo_adamw_step(const fo_tensor* t, int n_tensors, fo_format f, const fo_adamw_hparams* h,
                         void* stream)
 {
@@ -240,6 +269,7 @@ fo_status fo_adamw_step(const fo_tensor* t, int n_tensors, fo_format f, const fo
     sc.s[5] = (float)(1.0 / std::sqrt(bc2));
     sc.s[6] = (float)h->eps;
     sc.s[7] = (float)(1.0 - h->lr * h->weight_decay);
+    adamw_fast_bounds(sc);
     StepKernel k = pick_step<fo::kAdamW>(f);
     if (!k) return fail(FO_ERR_UNSUPPORTED, "format not provided");
     return launch_step(k, stage_smem(f), sc, t, n_tensors, (cudaStream_t)stream);
