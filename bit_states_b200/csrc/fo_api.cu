@@ -304,6 +304,22 @@ fo_status fo_sgdm_step(const fo_tensor* t, int n_tensors, fo_format f, const fo_
     return launch_step(k, stage_smem(f), sc, t, n_tensors, (cudaStream_t)stream);
 }
 
+fo_status fo_stream_copy(const fo_tensor* t, int n_tensors, fo_format f, int adamw_mix, void* stream)
+{
+    g_last_error.clear();
+    fo_status st = check_format(f);
+    if (st != FO_OK) return st;
+    st = check_tensors(t, n_tensors, f, adamw_mix != 0);
+    if (st != FO_OK) return st;
+    if (n_tensors == 0) return FO_OK;
+    fo::Scalars sc = {};
+    // the copy moves bytes only: the 16-bit formats do not matter, the ECC width does
+    StepKernel k;
+    if (adamw_mix) k = f.ecc_bits == 8 ? fo::step_kernel<0, 0, 8, fo::kCopyAdamW> : fo::step_kernel<0, 0, 16, fo::kCopyAdamW>;
+    else k = f.ecc_bits == 8 ? fo::step_kernel<0, 0, 8, fo::kCopySGDM> : fo::step_kernel<0, 0, 16, fo::kCopySGDM>;
+    return launch_step(k, stage_smem(f), sc, t, n_tensors, (cudaStream_t)stream);
+}
+
 fo_status fo_encode_master(const float* x32, void* w, void* ecc, int64_t n, fo_format f, void* stream)
 {
     g_last_error.clear();

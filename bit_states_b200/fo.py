@@ -48,7 +48,7 @@ class fo_format(ctypes.Structure):
     _fields_ = [("w_dtype", ctypes.c_int), ("grad_dtype", ctypes.c_int), ("ecc_bits", ctypes.c_int)]
 
 
-EXPORTS = ("fo_adamw_step", "fo_sgdm_step", "fo_encode_master", "fo_decode_master",
+EXPORTS = ("fo_adamw_step", "fo_sgdm_step", "fo_stream_copy", "fo_encode_master", "fo_decode_master",
            "fo_status_string", "fo_last_error", "fo_version")
 
 _lib = None
@@ -67,9 +67,10 @@ def load(path: str = LIB_PATH):
                                   ctypes.POINTER(fo_adamw_hparams), P]
     lib.fo_sgdm_step.argtypes = [ctypes.POINTER(fo_tensor), I, fo_format,
                                  ctypes.POINTER(fo_sgdm_hparams), P]
+    lib.fo_stream_copy.argtypes = [ctypes.POINTER(fo_tensor), I, fo_format, I, P]
     lib.fo_encode_master.argtypes = [P, P, P, I64, fo_format, P]
     lib.fo_decode_master.argtypes = [P, P, P, I64, fo_format, P]
-    for n in ("fo_adamw_step", "fo_sgdm_step", "fo_encode_master", "fo_decode_master"):
+    for n in ("fo_adamw_step", "fo_sgdm_step", "fo_stream_copy", "fo_encode_master", "fo_decode_master"):
         getattr(lib, n).restype = I
     lib.fo_status_string.argtypes = [I]
     lib.fo_status_string.restype = ctypes.c_char_p
@@ -140,6 +141,12 @@ def fo_adamw_step(descs, n_tensors: int, fmt: fo_format, h: fo_adamw_hparams, st
 def fo_sgdm_step(descs, n_tensors: int, fmt: fo_format, h: fo_sgdm_hparams, stream=None):
     _check(load().fo_sgdm_step(descs, n_tensors, fmt, ctypes.byref(h), _stream_handle(stream)),
            "fo_sgdm_step")
+
+
+def fo_stream_copy(descs, n_tensors: int, fmt: fo_format, adamw_mix: bool = True, stream=None):
+    """The step's byte traffic without its arithmetic (a bandwidth ceiling)."""
+    _check(load().fo_stream_copy(descs, n_tensors, fmt, int(bool(adamw_mix)), _stream_handle(stream)),
+           "fo_stream_copy")
 
 
 def fo_encode_master(x32, w, ecc, n: int, fmt: fo_format, stream=None):

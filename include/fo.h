@@ -148,6 +148,19 @@ FO_API fo_status fo_sgdm_step(const fo_tensor* t, int n_tensors, fo_format f,
                        const fo_sgdm_hparams* h, void* stream);
 
 /*
+ * fo_stream_copy - the byte traffic of one step without its arithmetic: reads
+ * every array fo_adamw_step (adamw_mix != 0) or fo_sgdm_step (adamw_mix == 0)
+ * reads and writes the same bytes back unchanged, through the same staging,
+ * work split and stores.  A measurement aid, not part of the method (the
+ * FlashOptim pages have no counterpart): its bandwidth is the practical
+ * ceiling for the step on the same tensors.  Arguments, validation and errors
+ * as fo_adamw_step / fo_sgdm_step; the 16-bit formats in f are not used, the
+ * ECC width is.  Concurrent calls or steps on the same tensors race.
+ */
+FO_API fo_status fo_stream_copy(const fo_tensor* t, int n_tensors, fo_format f, int adamw_mix,
+                        void* stream);
+
+/*
  * fo_encode_master - split n binary32 masters x32 (device) into the 16-bit
  * downcast w (round to nearest even) and the ECC codes ecc (device).
  * Used to wrap existing f32 weights and to import checkpoints.

@@ -1,0 +1,181 @@
+// fo_arith_check.cu - exhaustive / dense GPU checks of the identities the
+// step kernel's fast path relies on (test infrastructure, not the product).
+// Each check runs the kernel's own device functions (fo_kernels.cuh) against
+// the IEEE operation they replace and counts the inputs where the bits
+// differ.  Every kernel is a grid-stride loop over an index range; it writes
+// only to the counter / example arrays handed in by the host, at indices
+// below their stated sizes.
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "fo_kernels.cuh"
+
+namespace {
+
+__device__ __forceinline__ float rcp_full(float x)
+{
+    float r;
+    asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ float rsqrt_full(float x)
+{
+    float r;
+    asm("rsqrt.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ void note(unsigned long long* cnt, uint32_t* ex, int slot, uint32_t v)
+{
+    const unsigned long long k = atomicAdd(&cnt[slot], 1ull);
+    if (k < 4) ex[4 * slot + (int)k] = v;
+}
+
+// cnt[0]: rcp flush-to-zero form != full form with a normal full result
+// cnt[1]: rsqrt flush-to-zero form != full form
+// over every positive normal binary32
+__global__ void k_ftz(unsigned long long* cnt, uint32_t* ex)
+{
+    const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+    for (uint64_t i = 0x00800000ull + (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < 0x7F800000ull;
+         i += stride) {
+        const float x = __uint_as_float((uint32_t)i);
+        const float a = fo::rcp_approx(x), b = rcp_full(x);
+        if (__float_as_uint(a) != __float_as_uint(b) && fabsf(b) >= 1.17549435e-38f) note(cnt, ex, 0, (uint32_t)i);
+        if (__float_as_uint(fo::rsqrt_approx(x)) != __float_as_uint(rsqrt_full(x))) note(cnt, ex, 1, (uint32_t)i);
+    }
+}
+
+// cnt[0]: sqrt2_nr(v) != sqrt.rn(v) for v = +0 and every binary32 in (0, 2^64)
+// cnt[1]: sqrt2_nr(v) is not NaN for v in [2^64, inf]
+__global__ void k_sqrt(unsigned long long* cnt, uint32_t* ex)
+{
+    const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+    for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i <= 0x7F800000ull; i += 2 * stride) {
+        const uint32_t i0 = (uint32_t)i;
+        const uint32_t i1 = (uint32_t)(i + stride <= 0x7F800000ull ? i + stride : i);
+        const float2 v = make_float2(__uint_as_float(i0), __uint_as_float(i1));
+        const float2 s = fo::sqrt2_nr(v);
+        const uint32_t lim = 0x5F800000u;  // 2^64
+        if (i0 < lim) {
+            if (__float_as_uint(s.x) != __float_as_uint(__fsqrt_rn(v.x))) note(cnt, ex, 0, i0);
+        } else if (!isnan(s.x)) {
+            note(cnt, ex, 1, i0);
+        }
+        if (i1 < lim) {
+            if (__float_as_uint(s.y) != __float_as_uint(__fsqrt_rn(v.y))) note(cnt, ex, 0, i1);
+        } else if (!isnan(s.y)) {
+            note(cnt, ex, 1, i1);
+        }
+    }
+}
+
+__device__ __forceinline__ uint64_t splitmix(uint64_t z)
+{
+    z += 0x9E3779B97F4A7C15ull;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
+// cnt[0]: div2_nr(x, b) != div.rn(x, b) on n random pairs with b in
+// [2^-60, 2^20) and |x| in [2^-80, 2^61) (exponents uniform, significands
+// uniform), plus x = +0
+__global__ void k_div(uint64_t n, uint64_t seed, unsigned long long* cnt, uint32_t* ex)
+{
+    const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+    for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+        const uint64_t r = splitmix(seed ^ (i * 0xD1B54A32D192ED03ull));
+        const uint32_t eb = 127u - 60u + (uint32_t)((r >> 0) % 80u);    // 2^-60 .. 2^19
+        const uint32_t ea = 127u - 80u + (uint32_t)((r >> 8) % 141u);   // 2^-80 .. 2^60
+        const uint32_t mb = (uint32_t)(r >> 16) & 0x7FFFFFu;
+        const uint32_t ma = (uint32_t)(r >> 39) & 0x7FFFFFu;
+        const uint32_t sa = (uint32_t)(r >> 63) << 31;
+        float a = __uint_as_float(sa | (ea << 23) | ma);
+        if ((i & 1023u) == 0u) a = 0.0f;
+        const float b = __uint_as_float((eb << 23) | mb);
+        const float2 q = fo::div2_nr(make_float2(a, a), make_float2(b, b), make_float2(-b, -b));
+        if (__float_as_uint(q.x) != __float_as_uint(__fdiv_rn(a, b))) {
+            const unsigned long long k = atomicAdd(&cnt[0], 1ull);
+            if (k < 2) {
+                ex[2 * k] = __float_as_uint(a);
+                ex[2 * k + 1] = __float_as_uint(b);
+            }
+        }
+    }
+}
+
+// cnt[0]: largest ulp distance of rcp_approx(d) from RN(1/d) over every
+// binary32 d in [1, 2]; cnt[1]: scale_recips(S, S) != (1/S, 255/S) by div.rn
+// for every positive finite fp16 S (and S = 0 must give (0, 0)); cnt[2]:
+// v_code_value2 != RN(q / 255) by div.rn for a code q in [0, 255] (both byte
+// positions of a pair)
+__global__ void k_rcp_scales(unsigned long long* cnt, uint32_t* ex)
+{
+    const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+    for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i <= (1ull << 23); i += stride) {
+        const float d = __uint_as_float(0x3F800000u + (uint32_t)i);  // [1, 2]
+        const float r = fo::rcp_approx(d), e = __fdiv_rn(1.0f, d);
+        const int u = (int)__float_as_uint(r) - (int)__float_as_uint(e);
+        atomicMax(&cnt[0], (unsigned long long)(u < 0 ? -u : u));
+    }
+    for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < 256ull; i += stride) {
+        // both byte positions of a pair: codes i and 255 - i in bytes 2, 3 of the word
+        const uint32_t q0 = (uint32_t)i, q1 = 255u - (uint32_t)i;
+        const float2 v = fo::v_code_value2((q0 << 16) | (q1 << 24), 2u);
+        if (__float_as_uint(v.x) != __float_as_uint(__fdiv_rn((float)q0, 255.0f)) ||
+            __float_as_uint(v.y) != __float_as_uint(__fdiv_rn((float)q1, 255.0f)))
+            note(cnt, ex, 2, (uint32_t)i);
+        const float2 w = fo::v_code_value2(q0 | (q1 << 8), 0u);
+        if (__float_as_uint(w.x) != __float_as_uint(__fdiv_rn((float)q0, 255.0f)) ||
+            __float_as_uint(w.y) != __float_as_uint(__fdiv_rn((float)q1, 255.0f)))
+            note(cnt, ex, 2, (uint32_t)i);
+    }
+    for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < 0x7C00ull; i += stride) {
+        const float S = __half2float(__ushort_as_half((unsigned short)i));
+        const float2 q = fo::scale_recips(S, S);
+        const float e1 = S == 0.0f ? 0.0f : __fdiv_rn(1.0f, S), e2 = S == 0.0f ? 0.0f : __fdiv_rn(255.0f, S);
+        if (__float_as_uint(q.x) != __float_as_uint(e1) || __float_as_uint(q.y) != __float_as_uint(e2))
+            note(cnt, ex, 1, (uint32_t)i);
+    }
+}
+
+int launch_done(unsigned long long* hcnt, uint32_t* hex, unsigned long long* dcnt, uint32_t* dex)
+{
+    if (cudaGetLastError() != cudaSuccess) return 2;
+    if (cudaDeviceSynchronize() != cudaSuccess) return 3;
+    if (cudaMemcpy(hcnt, dcnt, 4 * sizeof(unsigned long long), cudaMemcpyDeviceToHost) != cudaSuccess) return 4;
+    if (cudaMemcpy(hex, dex, 16 * sizeof(uint32_t), cudaMemcpyDeviceToHost) != cudaSuccess) return 4;
+    return 0;
+}
+
+}  // namespace
+
+// which: 0 ftz forms, 1 square root, 2 division (n pairs, seed), 3 rcp bound
+// and scale reciprocals.  cnt: 4 counters, ex: 16 example words (host memory).
+extern "C" __attribute__((visibility("default"))) int fo_arith_check(int which, uint64_t n, uint64_t seed,
+                                                                     unsigned long long* cnt, uint32_t* ex)
+{
+    unsigned long long* dcnt = nullptr;
+    uint32_t* dex = nullptr;
+    if (cudaMalloc(&dcnt, 4 * sizeof(unsigned long long)) != cudaSuccess) return 1;
+    if (cudaMalloc(&dex, 16 * sizeof(uint32_t)) != cudaSuccess) {
+        cudaFree(dcnt);
+        return 1;
+    }
+    cudaMemset(dcnt, 0, 4 * sizeof(unsigned long long));
+    cudaMemset(dex, 0, 16 * sizeof(uint32_t));
+    const int grid = 148 * 8, block = 256;
+    switch (which) {
+    case 0: k_ftz<<<grid, block>>>(dcnt, dex); break;
+    case 1: k_sqrt<<<grid, block>>>(dcnt, dex); break;
+    case 2: k_div<<<grid, block>>>(n, seed, dcnt, dex); break;
+    case 3: k_rcp_scales<<<grid, block>>>(dcnt, dex); break;
+    default: break;
+    }
+    const int rc = launch_done(cnt, ex, dcnt, dex);
+    cudaFree(dcnt);
+    cudaFree(dex);
+    return rc;
+}

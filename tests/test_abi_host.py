@@ -146,3 +146,16 @@ def test_binding_raises_without_library(tmp_path):
             fo.load(str(tmp_path / "missing.so"))
     finally:
         fo._lib = saved
+
+
+def test_stream_copy_rejects_on_host(lib):
+    arr = (fo.fo_tensor * 1)(_t())
+    assert lib.fo_stream_copy(arr, 1, fo.fo_format(0, 0, 4), 1, None) == 2           # ECC width
+    assert lib.fo_stream_copy(None, 3, fo.make_format(), 1, None) == 1              # NULL table
+    odd = (fo.fo_tensor * 1)(_t(w=0x1001))
+    assert lib.fo_stream_copy(odd, 1, fo.make_format(), 1, None) == 3               # alignment
+    no_v = (fo.fo_tensor * 1)(_t(v_q=0, v_scale=0))
+    assert lib.fo_stream_copy(no_v, 1, fo.make_format(), 1, None) == 1              # AdamW mix needs v
+    assert lib.fo_stream_copy(arr, 0, fo.make_format(), 1, None) == 0               # no-op
+    assert lib.fo_stream_copy((fo.fo_tensor * 1)(_t(numel=0, w=0, ecc=0, grad=0, m_q=0, m_scale=0, v_q=0,
+                                                     v_scale=0)), 1, fo.make_format(), 0, None) == 0

@@ -1,0 +1,54 @@
+"""GPU checks of the arithmetic identities behind the step kernel's fast path
+(the kernel's own device functions, compiled with the library's flags, against
+the IEEE operations of the exact path):
+
+* the flush-to-zero approximate reciprocal / reciprocal square root equal the
+  full forms wherever the result is normal (every positive normal input);
+* the Newton-Raphson square root equals sqrt.rn on +0 and every binary32 in
+  (0, 2^64), and is NaN from 2^64 up (so the slice is redone exactly);
+* the Newton-Raphson quotient equals div.rn on 2^32 random pairs inside its
+  stated range (divisor in [2^-60, 2^20), numerator 0 or |x| in [2^-80, 2^61));
+* the approximate reciprocal is within 1 ulp of 1/d on [1, 2] (the bound the
+  compander's tie margin is derived from), the group-scale reciprocals
+  equal 1/S and 255/S by div.rn for every finite fp16 scale S >= 0, and the
+  computed variance-code values equal q/255 by div.rn for every code.
+"""
+import pytest
+import torch
+
+import arith_check
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    arith_check.build()
+    yield
+
+
+def test_flush_to_zero_forms_equal_full_forms_on_normals():
+    cnt, ex = arith_check.run(0)
+    assert cnt[0] == 0, f"rcp differs on {cnt[0]} inputs, e.g. {[hex(v) for v in ex[:4]]}"
+    assert cnt[1] == 0, f"rsqrt differs on {cnt[1]} inputs, e.g. {[hex(v) for v in ex[4:8]]}"
+
+
+def test_newton_raphson_sqrt_exhaustive():
+    cnt, ex = arith_check.run(1)
+    assert cnt[0] == 0, f"sqrt differs on {cnt[0]} inputs, e.g. {[hex(v) for v in ex[:4]]}"
+    assert cnt[1] == 0, f"not NaN on {cnt[1]} inputs >= 2^64, e.g. {[hex(v) for v in ex[4:8]]}"
+
+
+@pytest.mark.parametrize("seed", [1, 2])
+def test_newton_raphson_quotient_random_pairs(seed):
+    cnt, ex = arith_check.run(2, n=1 << 31, seed=seed)
+    assert cnt[0] == 0, f"quotient differs on {cnt[0]} pairs, e.g. {[hex(v) for v in ex[:4]]}"
+
+
+def test_reciprocal_bound_and_scale_reciprocals():
+    cnt, ex = arith_check.run(3)
+    assert cnt[0] <= 1, f"rcp.approx off by {cnt[0]} ulp on [1, 2]"
+    assert cnt[1] == 0, f"scale reciprocals differ for {cnt[1]} fp16 scales, e.g. {[hex(v) for v in ex[4:8]]}"
+    assert cnt[2] == 0, f"variance code values differ for {cnt[2]} codes, e.g. {ex[8:12]}"
