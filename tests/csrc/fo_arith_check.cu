@@ -141,6 +141,45 @@ __global__ void k_rcp_scales(unsigned long long* cnt, uint32_t* ex)
     }
 }
 
+// The fast 16-bit-master ECC8 codec of the step kernel against the exact one
+// (the device functions of the reference path), for W = bf16 (0) or fp16 (1):
+// cnt[0]: decode mismatches over every 16-bit pattern x' with every code in
+// [-127, 127] (pairs of elements, both lanes of a pair); cnt[1]: encode
+// mismatches (x' bits or code) over every binary32 x with |x| below the fast
+// path's limit (other x send the slice to the exact path).  Non-finite x'
+// are skipped for the decode, whose fast result is then caught downstream,
+// and so is a bf16 +-0 with an inward code, whose fast result must be out of
+// range.
+template <int W>
+__global__ void k_codec(unsigned long long* cnt, uint32_t* ex)
+{
+    const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+    for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (1ull << 16) * 128ull; i += stride) {
+        const uint32_t h = (uint32_t)(i >> 7), k = (uint32_t)(i & 127u);
+        if (fo::nonfinite16<W>(h)) continue;
+        // codes k and -k for the two lanes of the pair
+        const int r0 = (int)k, r1 = -(int)k;
+        uint32_t e[2] = {((uint32_t)r0 & 0xFFu) | (((uint32_t)r1 & 0xFFu) << 8), 0u};
+        const float2 x = fo::fast_decode_pair<W, 8>(h | (h << 16), e, 0);
+        const float e0 = fo::ecc_decode<W, 8>(h, r0), e1 = fo::ecc_decode<W, 8>(h, r1);
+        // bf16 +-0 with an inward code: the fast decode must land outside the
+        // fast path's range (the slice is then redone exactly)
+        const bool flagged1 = W == 0 && (h & 0x7FFFu) == 0u && r1 < 0;
+        const bool ok1 = flagged1 ? !(fabsf(x.y) < 3.39615136e38f) : __float_as_uint(x.y) == __float_as_uint(e1);
+        if (__float_as_uint(x.x) != __float_as_uint(e0) || !ok1) note(cnt, ex, 0, (uint32_t)i);
+    }
+    const uint32_t lim = W == 0 ? 0x7F7F8000u : 0x477FF000u;  // kDecodeLimit, 65520
+    for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (uint64_t)lim; i += stride) {
+        const float xa = __uint_as_float((uint32_t)i), xb = -xa;
+        int c0, c1;
+        const uint32_t wo = fo::fast_encode_pair<W, 8>(make_float2(xa, xb), c0, c1);
+        const uint32_t pa = fo::downcast16<W>(xa), pb = fo::downcast16<W>(xb);
+        if ((wo & 0xFFFFu) != pa || (wo >> 16) != pb || c0 != fo::ecc_encode<W, 8>(xa, pa) ||
+            c1 != fo::ecc_encode<W, 8>(xb, pb))
+            note(cnt, ex, 1, (uint32_t)i);
+    }
+}
+
 int launch_done(unsigned long long* hcnt, uint32_t* hex, unsigned long long* dcnt, uint32_t* dex)
 {
     if (cudaGetLastError() != cudaSuccess) return 2;
@@ -153,7 +192,7 @@ int launch_done(unsigned long long* hcnt, uint32_t* hex, unsigned long long* dcn
 }  // namespace
 
 // which: 0 ftz forms, 1 square root, 2 division (n pairs, seed), 3 rcp bound
-// and scale reciprocals.  cnt: 4 counters, ex: 16 example words (host memory).
+// and scale reciprocals, 4 / 5 fast bf16 / fp16 ECC8 codec.  cnt: 4 counters, ex: 16 example words (host memory).
 extern "C" __attribute__((visibility("default"))) int fo_arith_check(int which, uint64_t n, uint64_t seed,
                                                                      unsigned long long* cnt, uint32_t* ex)
 {
@@ -172,6 +211,8 @@ extern "C" __attribute__((visibility("default"))) int fo_arith_check(int which, 
     case 1: k_sqrt<<<grid, block>>>(dcnt, dex); break;
     case 2: k_div<<<grid, block>>>(n, seed, dcnt, dex); break;
     case 3: k_rcp_scales<<<grid, block>>>(dcnt, dex); break;
+    case 4: k_codec<0><<<grid, block>>>(dcnt, dex); break;
+    case 5: k_codec<1><<<grid, block>>>(dcnt, dex); break;
     default: break;
     }
     const int rc = launch_done(cnt, ex, dcnt, dex);

@@ -11,7 +11,11 @@ the IEEE operations of the exact path):
 * the approximate reciprocal is within 1 ulp of 1/d on [1, 2] (the bound the
   compander's tie margin is derived from), the group-scale reciprocals
   equal 1/S and 255/S by div.rn for every finite fp16 scale S >= 0, and the
-  computed variance-code values equal q/255 by div.rn for every code.
+  computed variance-code values equal q/255 by div.rn for every code;
+* the fast ECC8 codec of 16-bit masters (bit arithmetic; for fp16 an exact
+  fma at and below the smallest normal) equals the exact codec: decode of
+  every finite 16-bit pattern with every code, encode of every binary32 below
+  the fast path's limit (both signs).
 """
 import pytest
 import torch
@@ -52,3 +56,10 @@ def test_reciprocal_bound_and_scale_reciprocals():
     assert cnt[0] <= 1, f"rcp.approx off by {cnt[0]} ulp on [1, 2]"
     assert cnt[1] == 0, f"scale reciprocals differ for {cnt[1]} fp16 scales, e.g. {[hex(v) for v in ex[4:8]]}"
     assert cnt[2] == 0, f"variance code values differ for {cnt[2]} codes, e.g. {ex[8:12]}"
+
+
+@pytest.mark.parametrize("which,name", [(4, "bf16"), (5, "fp16")])
+def test_fast_ecc8_codec_exhaustive(which, name):
+    cnt, ex = arith_check.run(which)
+    assert cnt[0] == 0, f"{name} decode differs on {cnt[0]} (x', code) pairs, e.g. {[hex(v) for v in ex[:4]]}"
+    assert cnt[1] == 0, f"{name} encode differs on {cnt[1]} inputs, e.g. {[hex(v) for v in ex[4:8]]}"
