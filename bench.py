@@ -153,9 +153,11 @@ class ClockSampler:
         load = [s for s, p in zip(sm, pw) if p > 200.0] or sm
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower().startswith("active")})
+        pload = [p for p in pw if p > 200.0] or pw
         return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": max(mx) if mx else None,
                 "reasons": reasons, "samples": len(rows), "samples_under_load": len(load),
-                "power_w_max": max(pw) if pw else None}
+                "power_w_max": max(pw) if pw else None,
+                "power_w_median": statistics.median(pload) if pload else None}
 
 
 # ---------------------------------------------------------------------------
@@ -367,7 +369,7 @@ def main():
         total_ms, per_launch_ms = float(tt[0]), float(tt[1])
 
     # ---- the practical ceiling: the same byte mix without the arithmetic ----
-    ceiling_ms = None
+    ceiling_ms, ceiling_clocks = None, {}
     if args.launch_mode == "multi":
         def do_copy():
             fo.fo_stream_copy(descs, len(P.states), fmt, adam, stream)
@@ -377,6 +379,8 @@ def main():
         Kc = min(K, 50)
         cs = [torch.cuda.Event(enable_timing=True) for _ in range(Kc)]
         ce = [torch.cuda.Event(enable_timing=True) for _ in range(Kc)]
+        csampler = ClockSampler(gpu_id)
+        csampler.start()
         torch.cuda.synchronize()
         for k in range(Kc):
             if flush is not None:
@@ -385,6 +389,7 @@ def main():
             do_copy()
             ce[k].record(stream)
         torch.cuda.synchronize()
+        ceiling_clocks = csampler.stop()
         ceiling_ms = statistics.mean(cs[k].elapsed_time(ce[k]) for k in range(Kc))
         if dist:
             tc = torch.tensor([ceiling_ms], dtype=torch.float64, device=dev)
@@ -433,7 +438,8 @@ def main():
                           "stores, no arithmetic (after the timed region)",
                 "achieved": round(abytes / (ceiling_ms / 1e3) / 1e9, 1), "unit": "GB/s",
                 "frac_of_peak": round(abytes / (ceiling_ms / 1e3) / 1e9 / peak, 4),
-                "step_frac_of_ceiling": round(ceiling_ms / per_launch_ms, 4)},
+                "step_frac_of_ceiling": round(ceiling_ms / per_launch_ms, 4),
+                "clocks": {k: ceiling_clocks.get(k) for k in ("sm_mhz", "power_w_median", "power_w_max")}},
             "clocks": clocks,
             "gpu_launches": K * launches_per_step,
             "e2e": e2e,

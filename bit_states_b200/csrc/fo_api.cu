@@ -75,6 +75,7 @@ fo_status check_tensors(const fo_tensor* t, int n, const fo_format& f, bool adam
         char where[64];
         snprintf(where, sizeof where, "tensor %d: ", i);
         if (x.numel < 0) return fail(FO_ERR_INVALID_ARG, std::string(where) + "numel < 0");
+        if (x.numel > FO_MAX_NUMEL) return fail(FO_ERR_INVALID_ARG, std::string(where) + "numel > FO_MAX_NUMEL");
         if (x.numel == 0) continue;
         if (!x.w || !x.ecc || !x.grad || !x.m_q || !x.m_scale)
             return fail(FO_ERR_INVALID_ARG, std::string(where) + "NULL w / ecc / grad / m_q / m_scale");
@@ -175,9 +176,9 @@ fo_status launch_step(StepKernel k, int smem, const fo::Scalars& sc, const fo_te
             d.numel = x.numel;
             const uintptr_t a = (uintptr_t)x.w | (uintptr_t)x.grad | (uintptr_t)x.ecc | (uintptr_t)x.m_q |
                                 (uintptr_t)x.m_scale | (uintptr_t)x.v_q | (uintptr_t)x.v_scale;
-            d.aligned16 = (a & 15u) == 0 ? 1 : 0;
-            d.reserved = 0;
-            chunks += (x.numel + fo::kChunk - 1) / fo::kChunk;
+            d.n_chunks = (int32_t)((x.numel + fo::kChunk - 1) / fo::kChunk);
+            d.n_staged = (a & 15u) == 0 ? (int32_t)(x.numel / fo::kChunk) : 0;
+            chunks += d.n_chunks;
             P.chunk_start[++m] = chunks;
         }
         if (m == 0) break;

@@ -48,9 +48,9 @@
  *   - Kernel faults are asynchronous and surface at the caller's next
  *     synchronisation with the stream.
  *   - Alignment: 16-bit arrays need 2-byte alignment, int16 ECC arrays too.
- *     Any other alignment and any numel are accepted: tensors whose arrays
- *     are all 16-byte aligned take the vectorised path, others a scalar
- *     path inside the same kernel, with identical results.
+ *     Any other alignment and any numel up to FO_MAX_NUMEL are accepted:
+ *     tensors whose arrays are all 16-byte aligned take the vectorised path,
+ *     others a scalar path inside the same kernel, with identical results.
  *   - numel == 0 tensors are skipped; n_tensors == 0 is a no-op.
  *   - Results do not depend on the number of tensors per call, their order,
  *     or on whether they are stepped in one call or one call per tensor.
@@ -84,6 +84,10 @@ typedef enum { FO_DT_BF16 = 0, FO_DT_FP16 = 1 } fo_dtype;
 /* Largest n_tensors accepted by one call.  Calls with more tensors than fit
    one launch's parameter block are split into several launches. */
 #define FO_MAX_TENSORS_PER_CALL (1 << 20)
+
+/* Largest numel of one tensor (2^40 elements; larger ones are rejected with
+   FO_ERR_INVALID_ARG). */
+#define FO_MAX_NUMEL ((int64_t)1 << 40)
 
 /* One parameter tensor.  All pointers are device memory owned by the caller.
    Optimizer fields that a call does not use may be NULL (v_q / v_scale for

@@ -71,7 +71,7 @@ def _call_adamw(lib, tensors, fmt=None, hp=None, n=None):
 @pytest.mark.parametrize("case,status", [
     ("bad_wdt", 2), ("bad_ecc", 2), ("null_h", 1), ("step0", 1), ("beta1", 1), ("nan_lr", 1),
     ("neg_numel", 1), ("null_grad", 1), ("null_v", 1), ("odd_w", 3), ("odd_scale", 3),
-    ("odd_ecc16", 3), ("neg_n", 1), ("too_many", 4), ("null_array", 1),
+    ("odd_ecc16", 3), ("neg_n", 1), ("too_many", 4), ("null_array", 1), ("huge_numel", 1),
 ])
 def test_adamw_rejects_on_host(lib, case, status):
     t = [_t()]
@@ -88,6 +88,8 @@ def test_adamw_rejects_on_host(lib, case, status):
         hp = _hp(lr=float("nan"))
     elif case == "neg_numel":
         t = [_t(numel=-1)]
+    elif case == "huge_numel":
+        t = [_t(numel=(1 << 40) + 1)]
     elif case == "null_grad":
         t = [_t(grad=0)]
     elif case == "null_v":
