@@ -1,0 +1,156 @@
+"""Data-parallel sharded step on CPU ranks (gloo, world size 2): gradients
+reduce-scattered to the owners of their groups, each rank steps its slice of
+every bucket, the updated downcast weights all-gathered.  The bytes (the
+replicated x' on every rank, each rank's ECC / codes / scales) must equal one
+process stepping every tensor with the summed gradients.  The step on a rank
+is the oracle here (the GPU path passes the same slices to the fused kernel);
+the layout, the bucket slicing and the collectives are the code under test."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+from bit_states_b200.dp import GROUP, FlatLayout
+
+NUMELS = [100, 4096 + 7, 1, 3000, 33, 2048]
+HP = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01)
+BUCKET_GROUPS = 40
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _masters(ti, n):
+    from workloads import gen
+
+    return gen.normal(gen.stream_key(0, ti, 0, gen.KIND_MASTER), np.arange(n), 0.02)
+
+
+def _grads(rank, ti, t, n):
+    from workloads import gen
+
+    return gen.to_16bit(gen.normal(gen.stream_key(rank + 1, ti, t, gen.KIND_GRAD), np.arange(n), 1e-3), "bf16")
+
+
+def _flat(layout, per_tensor, dtype):
+    out = np.zeros(layout.numel, dtype)
+    for ti, a in enumerate(per_tensor):
+        o = layout.offsets[ti]
+        out[o:o + a.size] = a
+    return out
+
+
+def _oracle_step_fn(state, grad, t, stream):
+    import oracle
+
+    st = oracle.State(state.w.numpy().view(np.uint16), state.ecc.numpy(), state.m_q.numpy(),
+                      state.m_scale.numpy().view(np.uint16), state.v_q.numpy(),
+                      state.v_scale.numpy().view(np.uint16))
+    oracle.adamw_step(st, grad.numpy().view(np.uint16), **HP, step=t)
+
+
+def _worker(rank, world, port, q):
+    import torch
+    import torch.distributed as dist
+
+    import oracle
+    from bit_states_b200.dp import DataParallelStep, ShardedState
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        layout = FlatLayout(NUMELS, world, bucket_groups=BUCKET_GROUPS)
+        st = ShardedState(layout, rank, "cpu")
+        w, e = zip(*[oracle.encode_master(_masters(ti, n)) for ti, n in enumerate(NUMELS)])
+        wf, ef = _flat(layout, w, np.uint16), _flat(layout, e, np.int8)
+        st.w.copy_(torch.from_numpy(wf.view(np.int16)))
+        for s0, s1, go in st.slices:
+            st.ecc[go * GROUP:go * GROUP + (s1 - s0)] = torch.from_numpy(ef[s0:s1])
+        dp = DataParallelStep(st, step_fn=_oracle_step_fn, reduce_op="sum")
+        for t in (1, 2):
+            g = _flat(layout, [_grads(rank, ti, t, n) for ti, n in enumerate(NUMELS)], np.uint16)
+            dp.step(torch.from_numpy(g.view(np.int16)), t)
+        q.put((rank, st.w.numpy().copy(), st.ecc.numpy().copy(), st.m_q.numpy().copy(),
+               st.m_scale.numpy().copy(), st.v_q.numpy().copy(), st.v_scale.numpy().copy(),
+               list(st.slices)))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def _bf16_sum(a, b):
+    f = lambda u: (u.astype(np.uint32) << 16).view(np.float32)
+    s = f(a) + f(b)                       # one binary32 addition (exact for two bf16 values)
+    from workloads import gen
+
+    return gen.to_16bit(s.astype(np.float32), "bf16")
+
+
+def test_layout_buckets_cover_every_group_once():
+    for world in (1, 2, 3, 8):
+        L = FlatLayout(NUMELS, world, bucket_groups=BUCKET_GROUPS)
+        owned = []
+        for r in range(world):
+            for b in L.buckets:
+                g0, k = b.shard(world, r)
+                owned.extend(range(g0, g0 + k))
+        assert sorted(owned) == list(range(L.groups))
+        assert all(b.groups % world == 0 for b in L.buckets)
+        real = sum((n + 31) // 32 for n in NUMELS)
+        assert real <= L.groups < real + len(L.buckets) * world
+
+
+def test_two_rank_dp_step_equals_single_process():
+    import oracle
+
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = {}
+    for _ in range(2):
+        r = q.get(timeout=300)
+        res[r[0]] = r[1:]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    layout = FlatLayout(NUMELS, 2, bucket_groups=BUCKET_GROUPS)
+    # single-process reference: every tensor stepped with the summed gradients
+    exp = []
+    for ti, n in enumerate(NUMELS):
+        w, e = oracle.encode_master(_masters(ti, n))
+        st = oracle.State.zeros_like_master(w, e)
+        for t in (1, 2):
+            oracle.adamw_step(st, _bf16_sum(_grads(0, ti, t, n), _grads(1, ti, t, n)), **HP, step=t)
+        exp.append(st)
+    for rank in (0, 1):
+        w, ecc, mq, ms, vq, vs, slices = res[rank]
+        for ti, n in enumerate(NUMELS):
+            o = layout.offsets[ti]
+            assert np.array_equal(w[o:o + n].view(np.uint16), exp[ti].w), (rank, ti)
+        # owned groups: map back to (tensor, group)
+        for s0, s1, go in slices:
+            for g in range(s0 // GROUP, s1 // GROUP):
+                e0 = g * GROUP
+                ti = max(i for i in range(len(NUMELS)) if layout.offsets[i] <= e0)
+                lg = (e0 - layout.offsets[ti]) // GROUP
+                n = NUMELS[ti]
+                if lg * GROUP >= n:          # padding group
+                    continue
+                k = go + (g - s0 // GROUP)
+                a, b = lg * GROUP, min(n, lg * GROUP + GROUP)
+                L = b - a
+                assert np.array_equal(ecc[k * GROUP:k * GROUP + L], exp[ti].ecc[a:b]), (rank, ti, lg)
+                assert np.array_equal(mq[k * GROUP:k * GROUP + L], exp[ti].mq[a:b]), (rank, ti, lg)
+                assert np.array_equal(vq[k * GROUP:k * GROUP + L], exp[ti].vq[a:b]), (rank, ti, lg)
+                assert ms.view(np.uint16)[k] == exp[ti].ms[lg] and vs.view(np.uint16)[k] == exp[ti].vs[lg]
