@@ -455,36 +455,52 @@ def main():
 def run_e2e(args, wl, P, fmt, dev, dist, world, torch, fo):
     """Same metric through the public API with host buffers: every step
     copies each tensor's bf16 gradient from pinned host memory and reads the
-    updated downcast weights back to pinned host memory, per tensor in
-    gradient-release order, copies overlapped with the step kernels."""
-    from bit_states_b200.state import CompressedAdamW
+    updated downcast weights back to pinned host memory, in gradient-release
+    order.  Tensors are cut at group boundaries into pieces of at most
+    PIECE elements, so that the host-to-device copies, the step launches and
+    the device-to-host copies of consecutive pieces overlap (a ring of stage
+    buffers on the device, one stream per copy direction)."""
+    from bit_states_b200.fo import TensorState
 
     if wl.optimizer != "adamw":
         return None
-    opt = CompressedAdamW(P, lr=wl.hparams["lr"], betas=(wl.hparams["beta1"], wl.hparams["beta2"]),
-                          eps=wl.hparams["eps"], weight_decay=wl.hparams["weight_decay"], grad_dtype=wl.grad_dtype)
     from workloads import device as wdev
 
-    big = max(P.numels)
-    stage = [torch.empty(big, dtype=torch.int16, device=dev) for _ in range(2)]
-    # host gradients: the largest tensor's synthetic gradient, reused as the
-    # source of every tensor's copy (the bytes moved are the full list's)
-    wdev.grad_16(wl, int(np.argmax(P.numels)), 1, stage[0])
-    host_g = torch.empty(big, dtype=torch.int16, pin_memory=True)
-    host_g.copy_(stage[0])
-    host_w = torch.empty(big, dtype=torch.int16, pin_memory=True)
+    PIECE, RING = 1 << 24, 4
+    pieces = []                            # (tensor, first element, elements), release order
+    for ti in list(range(len(P.numels)))[::-1]:
+        n = P.numels[ti]
+        for e0 in range(0, n, PIECE):
+            pieces.append((ti, e0, min(PIECE, n - e0)))
+    stage = [torch.empty(PIECE, dtype=torch.int16, device=dev) for _ in range(RING)]
+    # host gradient: a synthetic gradient piece, the source of every piece's
+    # copy (the bytes moved are the full list's)
+    big = int(np.argmax(P.numels))
+    tmp = torch.empty(P.numels[big], dtype=torch.int16, device=dev)
+    wdev.grad_16(wl, big, 1, tmp)
+    host_g = torch.empty(PIECE, dtype=torch.int16, pin_memory=True)
+    host_g.copy_(tmp[:PIECE])
+    del tmp
+    host_w = torch.empty(PIECE, dtype=torch.int16, pin_memory=True)
     s_in = torch.cuda.Stream(dev)
     s_out = torch.cuda.Stream(dev)
     comp = torch.cuda.current_stream(dev)
-    order = list(range(len(P.numels)))[::-1]
     h2d = sum(P.numels) * 2
     d2h = sum(P.numels) * 2
+    h = wl.hparams
+    descs = []
+    for ti, e0, n in pieces:
+        st = P.states[ti]
+        g0, g1 = e0 // 32, (e0 + n + 31) // 32
+        sub = TensorState(st.w[e0:e0 + n], st.ecc[e0:e0 + n], st.m_q[e0:e0 + n], st.m_scale[g0:g1],
+                          st.v_q[e0:e0 + n], st.v_scale[g0:g1])
+        descs.append((sub, n))
 
     def one_step(t):
-        done = [None, None]
-        for j, ti in enumerate(order):
-            n = P.numels[ti]
-            b = j % 2
+        hp = fo.fo_adamw_hparams(h["lr"], h["beta1"], h["beta2"], h["eps"], h["weight_decay"], t)
+        done = [None] * RING
+        for j, (sub, n) in enumerate(descs):
+            b = j % RING
             with torch.cuda.stream(s_in):
                 if done[b] is not None:
                     s_in.wait_event(done[b])
@@ -492,13 +508,13 @@ def run_e2e(args, wl, P, fmt, dev, dist, world, torch, fo):
                 ev_in = torch.cuda.Event()
                 ev_in.record(s_in)
             comp.wait_event(ev_in)
-            opt.step_tensor(ti, stage[b][:n], t, comp)
+            fo.fo_adamw_step(fo.descriptors([sub], [stage[b][:n]]), 1, fmt, hp, comp)
             ev_done = torch.cuda.Event()
             ev_done.record(comp)
             done[b] = ev_done
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_done)
-                host_w[:n].copy_(P.states[ti].w, non_blocking=True)
+                host_w[:n].copy_(sub.w, non_blocking=True)
         comp.wait_stream(s_out)
         comp.wait_stream(s_in)
 
@@ -523,8 +539,10 @@ def run_e2e(args, wl, P, fmt, dev, dist, world, torch, fo):
     value = world * sum(P.numels) * K / (ms / 1e3) / 1e9
     return {"value": round(value, 3), "unit": "Gparams/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(ms / K, 3), "steps": K,
-            "how": "per tensor: pinned-host bf16 grad -> device (copy stream), fo_adamw_step, updated bf16 "
-                   "weights -> pinned host (copy stream); double-buffered, overlapped"}
+            "how": f"tensors cut into group-aligned pieces of <= {PIECE} params in gradient-release order; per "
+                   "piece: pinned-host bf16 grad -> device (copy stream), fo_adamw_step, updated bf16 weights -> "
+                   f"pinned host (copy stream); {RING} device stage buffers, copies overlapped with the steps",
+            "launches_per_step": len(descs)}
 
 
 if __name__ == "__main__":
