@@ -216,6 +216,18 @@ def time_oracle(wl, n_params: int, steps: int, warmup: int, threads: int):
     return n * steps / dt / 1e9, dt, n
 
 
+def arm_config(wl, args, world):
+    """The workload description both arms print."""
+    abytes = algorithmic_bytes(wl)
+    return {"workload": f"{wl.name}: {len(wl.tensors)} tensors, {wl.numel} params per GPU, "
+                        f"{wl.optimizer} {wl.w_dtype}+ecc{wl.ecc_bits}, int8/uint8 companded states",
+            "launch": "one multi-tensor launch per step" if args.launch_mode == "multi" else
+                      f"{len(wl.tensors)} per-tensor launches per step (gradient release order)",
+            "l2": ("L2 flushed (512 MB write) before every step; steps timed alone" if args.flush_l2 else
+                   "inputs larger than L2 (%.2f GB per step vs 126 MB)" % (abytes / 1e9)),
+            "parallelism": f"weak-scaling shards x{world}, no data-path collective"}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
@@ -234,8 +246,7 @@ def run_reference(args, rank, world):
             "n_gpus": args.gpus, "steps": steps, "warmup": min(args.warmup, 3),
             "ms_per_step": round(dt / steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": wl.name, "params": wl.numel, "sampled_params_per_step": n,
-                       "optimizer": wl.optimizer, "format": f"{wl.w_dtype}+ecc{wl.ecc_bits}"},
+            "config": arm_config(wl, args, world),
             "cpu_baseline": {"value": round(value, 6), "unit": "Gparams/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(value, 6), "unit": "Gparams/s", "h2d_bytes_per_step": 0,
@@ -422,13 +433,7 @@ def main():
             "metric": METRIC, "value": round(value, 3), "unit": "Gparams/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": round(total_ms / K, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": f"{wl.name}: {len(wl.tensors)} tensors, {n_params} params per GPU, "
-                                   f"{wl.optimizer} {wl.w_dtype}+ecc{wl.ecc_bits}, int8/uint8 companded states",
-                       "launch": "one multi-tensor launch per step" if args.launch_mode == "multi" else
-                                 f"{len(order)} per-tensor launches per step (gradient release order)",
-                       "l2": ("L2 flushed (512 MB write) before every step; steps timed alone" if args.flush_l2 else
-                              "inputs larger than L2 (%.2f GB per step vs 126 MB)" % (abytes / 1e9)),
-                       "parallelism": f"weak-scaling shards x{world}, no data-path collective"},
+            "config": arm_config(wl, args, world),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic,
                          "peak_kind": peak_kind, "algorithmic_bytes_per_launch": abytes,
