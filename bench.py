@@ -260,6 +260,8 @@ def run_reference(args, rank, world):
 
 def main():
     args = parse()
+    if args.config.endswith("-release"):
+        args.launch_mode = "release"  # the gradient-release workload is one call per tensor
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
