@@ -85,10 +85,17 @@ def measured_peaks():
 
 
 def kernel_source_sha() -> str:
+    """Hash of the kernel sources' code (comments and whitespace removed), so
+    that a profile stays attached to the code it measured."""
+    import re
+
     h = hashlib.sha256()
     for f in ("fo_codec.cuh", "fo_kernels.cuh", "fo_api.cu"):
-        with open(os.path.join(ROOT, "bit_states_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "bit_states_b200", "csrc", f)) as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        h.update(" ".join(src.split()).encode())
     return h.hexdigest()[:16]
 
 
