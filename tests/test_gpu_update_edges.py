@@ -90,9 +90,10 @@ HP_CASES = {
 }
 
 
+@pytest.mark.parametrize("nbits", [8, 16])
 @pytest.mark.parametrize("wdt", ["bf16", "fp16"])
 @pytest.mark.parametrize("hp_name", list(HP_CASES))
-def test_update_edges_every_byte(wdt, hp_name):
+def test_update_edges_every_byte(wdt, hp_name, nbits):
     hp = HP_CASES[hp_name]
     rng = np.random.default_rng(20 + len(hp_name))
     blocks = _blocks(rng, wdt)
@@ -100,25 +101,25 @@ def test_update_edges_every_byte(wdt, hp_name):
     x = np.concatenate([b[0] for b in blocks] + [(rng.standard_normal(tail) * 0.02).astype(np.float32)])
     n = x.size
     wcode = 0 if wdt == "bf16" else 1
-    w, e = oracle.encode_master(x, wcode, 8)
+    w, e = oracle.encode_master(x, wcode, nbits)
     st = oracle.State.zeros_like_master(w, e)
     ng = (n + 31) // 32
     wv = torch.from_numpy(w.view(np.int16).copy()).to(DEV)
-    ev = torch.from_numpy(e.copy()).to(DEV)
+    ev = torch.from_numpy(e.copy()).to(DEV)  # int8 or int16 codes
     mqv = torch.zeros(n, dtype=torch.int8, device=DEV)
     vqv = torch.zeros(n, dtype=torch.uint8, device=DEV)
     msv = torch.zeros(ng, dtype=torch.int16, device=DEV)
     vsv = torch.zeros(ng, dtype=torch.int16, device=DEV)
     gv = torch.zeros(n, dtype=torch.int16, device=DEV)
     dst = fo.TensorState(wv, ev, mqv, msv, vqv, vsv)
-    fmt = fo.make_format(wdt, "bf16", 8)
+    fmt = fo.make_format(wdt, "bf16", nbits)
     for t in range(1, 4):
         r = np.random.default_rng(1000 * t + len(hp_name))
         g32 = np.concatenate([b[1](r) for b in blocks] + [(r.standard_normal(tail) * 1e-3).astype(np.float32)])
         gb = gen.to_16bit(g32.astype(np.float32), "bf16")
         gv.copy_(torch.from_numpy(gb.view(np.int16)))
         fo.fo_adamw_step(fo.descriptors([dst], [gv]), 1, fmt, fo.fo_adamw_hparams(**hp, step=t))
-        oracle.adamw_step(st, gb, **hp, step=t, wdt=wcode, gdt=0, ecc_bits=8)
+        oracle.adamw_step(st, gb, **hp, step=t, wdt=wcode, gdt=0, ecc_bits=nbits)
         torch.cuda.synchronize()
         for name, got, exp in (("w", U.to_np_bytes(wv), st.w.view(np.uint16)),
                                ("ecc", ev.cpu().numpy(), st.ecc),
