@@ -105,6 +105,23 @@ class ShardedState:
             self.slices.append((g0 * GROUP, (g0 + k) * GROUP, o))
             o += k
 
+    def encode_from(self, x32_flat, fmt, group=None, w_dtype: str = "bf16"):
+        """Initialise from f32 masters in the flat layout (every rank passes
+        the same values): each rank encodes the groups it owns (downcast and
+        ECC), then the downcast weights are all-gathered."""
+        import torch
+        import torch.distributed as dist
+
+        from . import fo
+
+        wflat = self.w.view({"bf16": torch.bfloat16, "fp16": torch.float16}[w_dtype])
+        for bi, b in enumerate(self.layout.buckets):
+            s0, s1, go = self.slices[bi]
+            n, o = s1 - s0, go * GROUP
+            fo.fo_encode_master(x32_flat[s0:s1], self.w[s0:s1], self.ecc[o:o + n], n, fmt)
+            e0 = b.g0 * GROUP
+            dist.all_gather_into_tensor(wflat[e0:e0 + b.groups * GROUP], wflat[s0:s1], group=group)
+
     def bucket_state(self, bi: int):
         """TensorState of this rank's slice of bucket bi (one flat tensor)."""
         from .fo import TensorState

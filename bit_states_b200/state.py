@@ -69,6 +69,23 @@ class CompressedParams:
             t += self.v_q.nbytes + self.v_scale.nbytes
         return t
 
+    def state_dict(self) -> dict:
+        """Checkpoint: the compressed arrays (the masters are their downcast +
+        ECC, so nothing is lost) and the layout they were allocated with."""
+        d = {"numels": list(self.numels), "adam": self.adam, "ecc_bits": self.ecc_bits, "w_dtype": self.w_dtype,
+             "w": self.w, "ecc": self.ecc, "m_q": self.m_q, "m_scale": self.m_scale}
+        if self.adam:
+            d["v_q"], d["v_scale"] = self.v_q, self.v_scale
+        return d
+
+    def load_state_dict(self, d: dict) -> None:
+        """Resume from state_dict(): the same parameter list and format."""
+        if (list(d["numels"]) != self.numels or bool(d["adam"]) != self.adam or int(d["ecc_bits"]) != self.ecc_bits
+                or d["w_dtype"] != self.w_dtype):
+            raise ValueError("checkpoint was taken with another parameter list or format")
+        for k in ("w", "ecc", "m_q", "m_scale") + (("v_q", "v_scale") if self.adam else ()):
+            getattr(self, k).copy_(d[k])
+
     def encode_from(self, i: int, x32, stream=None):
         """Split f32 masters of tensor i into downcast + ECC (device kernel)."""
         st = self.states[i]
@@ -84,7 +101,8 @@ class CompressedParams:
 class CompressedAdamW:
     """AdamW over a parameter list with bf16/fp16 + ECC masters and 8-bit
     companded states; ``step`` is one fused kernel launch for the whole list
-    (or one per call when used for gradient release)."""
+    (or one per call when used for gradient release).  A checkpoint is the
+    parameters' state_dict() plus this optimizer's step count ``t``."""
 
     def __init__(self, params: CompressedParams, lr=1e-3, betas=(0.9, 0.999), eps=1e-8,
                  weight_decay=0.01, grad_dtype="bf16"):

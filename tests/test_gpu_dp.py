@@ -57,11 +57,12 @@ def test_dp_step_one_rank_equals_fused_step(pg):
                           torch.zeros((n + 31) // 32, dtype=torch.int16, device=dev),
                           torch.zeros(n, dtype=torch.uint8, device=dev),
                           torch.zeros((n + 31) // 32, dtype=torch.int16, device=dev)) for n in NUMELS]
+    x32 = torch.zeros(layout.numel, dtype=torch.float32, device=dev)
     for ti, (n, x) in enumerate(zip(NUMELS, xs)):
         xd = torch.from_numpy(x).to(dev)
         fo.fo_encode_master(xd, ref[ti].w, ref[ti].ecc, n, fmt)
-        o = layout.offsets[ti]
-        fo.fo_encode_master(xd, st.w[o:o + n], st.ecc[o:o + n], n, fmt)   # world 1: every group owned
+        layout.tensor_view(x32, ti).copy_(xd)
+    st.encode_from(x32, fmt)
     for t in (1, 2, 3):
         gs = [torch.from_numpy(gen.to_16bit(gen.normal(gen.stream_key(0, ti, t, gen.KIND_GRAD), np.arange(n), 1e-3),
                                             "bf16").view(np.int16)).to(dev) for ti, n in enumerate(NUMELS)]
