@@ -7,4 +7,4 @@ binding and ``state`` allocates the compressed buffers with torch.
 from . import fo  # noqa: F401
 from .fo import (FoError, TensorState, descriptors, fo_adamw_hparams, fo_adamw_step,  # noqa: F401
                  fo_decode_master, fo_encode_master, fo_format, fo_sgdm_hparams, fo_sgdm_step,
-                 fo_tensor, make_format)
+                 fo_stream_copy, fo_tensor, make_format)

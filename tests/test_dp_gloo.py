@@ -9,7 +9,6 @@ import os
 import socket
 
 import numpy as np
-import pytest
 import torch.multiprocessing as mp
 
 from bit_states_b200.dp import GROUP, FlatLayout

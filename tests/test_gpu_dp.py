@@ -4,7 +4,6 @@ world-size-1 NCCL group, so the collectives are copies and no rank waits on
 another.  Its bytes must equal one fused multi-tensor step on the same
 tensors.  (Two or more GPUs are not available here; the exchange between ranks
 is covered on CPU by tests/test_dp_gloo.py.)"""
-import os
 import socket
 
 import numpy as np
@@ -15,7 +14,6 @@ from bit_states_b200 import fo
 from bit_states_b200.dp import GROUP, DataParallelStep, FlatLayout, ShardedState
 from workloads import gen
 
-import gpu_util as U
 
 pytestmark = pytest.mark.gpu
 

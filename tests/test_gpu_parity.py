@@ -11,7 +11,6 @@ import torch
 
 import oracle
 from bit_states_b200 import fo
-from bit_states_b200.state import CompressedParams
 from workloads import gen, workload
 from workloads import device as wdev
 from workloads.shapes import TensorSpec, Workload, ADAMW_HP, SGDM_HP

@@ -16,7 +16,6 @@ What fixes the expected values independently of the oracle:
   * "within one quantisation step" for heavy-tailed random data.
 """
 import numpy as np
-import pytest
 import torch
 
 M, V, VSQRT = 0, 1, 2

@@ -6,7 +6,6 @@ import os
 import socket
 
 import numpy as np
-import pytest
 import torch.multiprocessing as mp
 
 from bit_states_b200.shard import GROUP, shard_spans
