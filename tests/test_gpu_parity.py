@@ -166,6 +166,17 @@ def test_ragged_multitensor_all_formats(opt, wdt, gdt, nbits):
     _run_full_compare(wl, 3)
 
 
+@pytest.mark.parametrize("hp", [
+    dict(lr=3e-4, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1),     # LLM-style betas
+    dict(lr=1e-2, beta1=0.8, beta2=0.99, eps=1e-6, weight_decay=0.0),     # no decay: x (1 - lr wd) = x
+    dict(lr=1e-3, beta1=0.0, beta2=0.999, eps=1e-12, weight_decay=0.01),  # no momentum averaging
+])
+def test_ragged_adamw_hyperparameter_sets(hp):
+    wl = _ragged_workload("adamw", "bf16", "bf16", 8)
+    wl.hparams = dict(hp)
+    _run_full_compare(wl, 3)
+
+
 @pytest.mark.parametrize("nesterov,damp", [(1, 0.0), (0, 0.25)])
 def test_sgdm_variants(nesterov, damp):
     wl = _ragged_workload("sgdm", "fp16", "fp16", 8)
@@ -234,6 +245,19 @@ def test_empty_and_tiny_tensors_in_one_call():
         o.step(1)
         exp = o.expected()
         assert all(v == 0 for v in U.mismatches(exp, U.gather_device(P, ti, exp)).values())
+
+
+def test_many_tensors_split_across_launches():
+    """1000 tensors in one call: more than one launch's parameter block holds
+    (384 descriptors), so the call is split into several launches.  Every
+    byte of every tensor against the oracle."""
+    rng = np.random.default_rng(17)
+    sizes = [int(v) for v in rng.integers(1, 2600, 1000)]
+    for i in range(0, 1000, 97):
+        sizes[i] = 512 * int(rng.integers(1, 4))      # whole chunks: the staged path
+    wl = _ragged_workload("adamw", "bf16", "bf16", 8)
+    wl.tensors = [TensorSpec(f"t{i}", (n,), "normal", 0.02) for i, n in enumerate(sizes)]
+    _run_full_compare(wl, 2)
 
 
 # ---- gradient release == one multi-tensor launch -------------------------------------
