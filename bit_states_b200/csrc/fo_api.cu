@@ -92,15 +92,31 @@ fo_status check_tensors(const fo_tensor* t, int n, const fo_format& f, bool adam
 
 using StepKernel = void (*)(const fo::StepParams);
 
+// one step kernel with its launch geometry (fo::Geometry)
+struct StepLaunch {
+    StepKernel k;
+    int threads;    // threads per block
+    int smem;       // dynamic shared memory per block (stage buffers)
+    int64_t chunk;  // elements per chunk
+};
+
+template <int WDT, int GDT, int NB, int KIND>
+StepLaunch step_launch()
+{
+    using G = fo::Geometry<NB, KIND>;
+    return {fo::step_kernel<WDT, GDT, NB, KIND>, G::kBlockThreads, fo::step_smem_bytes<NB, KIND>(), G::kChunk};
+}
+
+// the step kernel of a format (k = nullptr if the format is not provided)
 template <int KIND>
-StepKernel pick_step(const fo_format& f)
+StepLaunch pick_step(const fo_format& f)
 {
 #define FO_PICK(W, G, N)                                                                  \
-    if (f.w_dtype == W && f.grad_dtype == G && f.ecc_bits == N) return fo::step_kernel<W, G, N, KIND>;
+    if (f.w_dtype == W && f.grad_dtype == G && f.ecc_bits == N) return step_launch<W, G, N, KIND>();
     FO_PICK(0, 0, 8) FO_PICK(0, 1, 8) FO_PICK(1, 0, 8) FO_PICK(1, 1, 8)
     FO_PICK(0, 0, 16) FO_PICK(0, 1, 16) FO_PICK(1, 0, 16) FO_PICK(1, 1, 16)
 #undef FO_PICK
-    return nullptr;
+    return {nullptr, 0, 0, 0};
 }
 
 struct LaunchCache {
@@ -113,7 +129,7 @@ struct LaunchCache {
 
 // once per (device, kernel): allow the dynamic shared memory of the stage
 // buffers and find how many blocks fit on one SM
-fo_status prepare_kernel(StepKernel k, int smem, int* blocks_per_sm)
+fo_status prepare_kernel(StepKernel k, int threads, int smem, int* blocks_per_sm)
 {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -127,7 +143,7 @@ fo_status prepare_kernel(StepKernel k, int smem, int* blocks_per_sm)
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
     int b = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, k, fo::kThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, k, threads, smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
     if (b < 1) b = 1;
     if (g_launch.n < 128) {
@@ -140,9 +156,10 @@ fo_status prepare_kernel(StepKernel k, int smem, int* blocks_per_sm)
     return FO_OK;
 }
 
-fo_status launch_step(StepKernel k, int smem, const fo::Scalars& sc, const fo_tensor* t, int n,
-                      cudaStream_t stream)
+fo_status launch_step(const StepLaunch& L, const fo::Scalars& sc, const fo_tensor* t, int n, cudaStream_t stream)
 {
+    const int64_t chunk = L.chunk;
+    const int warps = L.threads / 32;
     bool any = false;
     for (int j = 0; j < n && !any; j++) any = t[j].numel > 0;
     if (!any) return FO_OK;
@@ -150,7 +167,7 @@ fo_status launch_step(StepKernel k, int smem, const fo::Scalars& sc, const fo_te
     fo_status st = device_sms(&sms);
     if (st != FO_OK) return st;
     int bps = 1;
-    st = prepare_kernel(k, smem, &bps);
+    st = prepare_kernel(L.k, L.threads, L.smem, &bps);
     if (st != FO_OK) return st;
     // kernel parameters are copied at launch, so one block of host memory
     // per thread serves every launch
@@ -176,8 +193,8 @@ fo_status launch_step(StepKernel k, int smem, const fo::Scalars& sc, const fo_te
             d.numel = x.numel;
             const uintptr_t a = (uintptr_t)x.w | (uintptr_t)x.grad | (uintptr_t)x.ecc | (uintptr_t)x.m_q |
                                 (uintptr_t)x.m_scale | (uintptr_t)x.v_q | (uintptr_t)x.v_scale;
-            d.n_chunks = (int32_t)((x.numel + fo::kChunk - 1) / fo::kChunk);
-            d.n_staged = (a & 15u) == 0 ? (int32_t)(x.numel / fo::kChunk) : 0;
+            d.n_chunks = (int32_t)((x.numel + chunk - 1) / chunk);
+            d.n_staged = (a & 15u) == 0 ? (int32_t)(x.numel / chunk) : 0;
             chunks += d.n_chunks;
             P.chunk_start[++m] = chunks;
         }
@@ -186,10 +203,10 @@ fo_status launch_step(StepKernel k, int smem, const fo::Scalars& sc, const fo_te
         P.total_chunks = chunks;
         // a sentinel past the last tensor keeps the device-side walk bounded
         for (int j = m + 1; j <= fo::kMaxTensorsPerLaunch; j++) P.chunk_start[j] = INT64_MAX;
-        int64_t grid = (chunks + fo::kWarps - 1) / fo::kWarps;
+        int64_t grid = (chunks + warps - 1) / warps;
         const int64_t cap = (int64_t)sms * bps;
         if (grid > cap) grid = cap;
-        k<<<(unsigned)grid, fo::kThreads, smem, stream>>>(P);
+        L.k<<<(unsigned)grid, L.threads, L.smem, stream>>>(P);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "step kernel launch");
     }
@@ -197,11 +214,6 @@ fo_status launch_step(StepKernel k, int smem, const fo::Scalars& sc, const fo_te
 }
 
 bool is_finite(double v) { return std::isfinite(v); }
-
-int stage_smem(const fo_format& f)
-{
-    return f.ecc_bits == 8 ? fo::step_smem_bytes<8>() : fo::step_smem_bytes<16>();
-}
 
 int64_t grid_for(int64_t n, int sms)
 {
@@ -271,9 +283,9 @@ fo_status fo_adamw_step(const fo_tensor* t, int n_tensors, fo_format f, const fo
     sc.s[6] = (float)h->eps;
     sc.s[7] = (float)(1.0 - h->lr * h->weight_decay);
     adamw_fast_bounds(sc);
-    StepKernel k = pick_step<fo::kAdamW>(f);
-    if (!k) return fail(FO_ERR_UNSUPPORTED, "format not provided");
-    return launch_step(k, stage_smem(f), sc, t, n_tensors, (cudaStream_t)stream);
+    const StepLaunch L = pick_step<fo::kAdamW>(f);
+    if (!L.k) return fail(FO_ERR_UNSUPPORTED, "format not provided");
+    return launch_step(L, sc, t, n_tensors, (cudaStream_t)stream);
 }
 
 fo_status fo_sgdm_step(const fo_tensor* t, int n_tensors, fo_format f, const fo_sgdm_hparams* h,
@@ -300,9 +312,9 @@ fo_status fo_sgdm_step(const fo_tensor* t, int n_tensors, fo_format f, const fo_
     sc.s[5] = h->step == 1 ? 1.0f : 0.0f;
     sc.s[6] = 0.0f;
     sc.s[7] = 0.0f;
-    StepKernel k = pick_step<fo::kSGDM>(f);
-    if (!k) return fail(FO_ERR_UNSUPPORTED, "format not provided");
-    return launch_step(k, stage_smem(f), sc, t, n_tensors, (cudaStream_t)stream);
+    const StepLaunch L = pick_step<fo::kSGDM>(f);
+    if (!L.k) return fail(FO_ERR_UNSUPPORTED, "format not provided");
+    return launch_step(L, sc, t, n_tensors, (cudaStream_t)stream);
 }
 
 fo_status fo_stream_copy(const fo_tensor* t, int n_tensors, fo_format f, int adamw_mix, void* stream)
@@ -315,10 +327,10 @@ fo_status fo_stream_copy(const fo_tensor* t, int n_tensors, fo_format f, int ada
     if (n_tensors == 0) return FO_OK;
     fo::Scalars sc = {};
     // the copy moves bytes only: the 16-bit formats do not matter, the ECC width does
-    StepKernel k;
-    if (adamw_mix) k = f.ecc_bits == 8 ? fo::step_kernel<0, 0, 8, fo::kCopyAdamW> : fo::step_kernel<0, 0, 16, fo::kCopyAdamW>;
-    else k = f.ecc_bits == 8 ? fo::step_kernel<0, 0, 8, fo::kCopySGDM> : fo::step_kernel<0, 0, 16, fo::kCopySGDM>;
-    return launch_step(k, stage_smem(f), sc, t, n_tensors, (cudaStream_t)stream);
+    StepLaunch L;
+    if (adamw_mix) L = f.ecc_bits == 8 ? step_launch<0, 0, 8, fo::kCopyAdamW>() : step_launch<0, 0, 16, fo::kCopyAdamW>();
+    else L = f.ecc_bits == 8 ? step_launch<0, 0, 8, fo::kCopySGDM>() : step_launch<0, 0, 16, fo::kCopySGDM>();
+    return launch_step(L, sc, t, n_tensors, (cudaStream_t)stream);
 }
 
 fo_status fo_encode_master(const float* x32, void* w, void* ecc, int64_t n, fo_format f, void* stream)

@@ -148,7 +148,7 @@ def test_flat_1m_ten_adamw_steps_every_byte():
 
 # ---- ragged sizes, misaligned views, all formats ------------------------------------
 
-RAGGED = [1, 2, 31, 32, 33, 255, 256, 257, 511, 512, 513, 1000, 4095, 4096, 65537]
+RAGGED = [1, 2, 31, 32, 33, 255, 256, 257, 511, 512, 513, 767, 768, 769, 1000, 1536, 1537, 4095, 4096, 65537]
 
 
 def _ragged_workload(opt, wdt, gdt, nbits):
@@ -254,7 +254,7 @@ def test_many_tensors_split_across_launches():
     rng = np.random.default_rng(17)
     sizes = [int(v) for v in rng.integers(1, 2600, 1000)]
     for i in range(0, 1000, 97):
-        sizes[i] = 512 * int(rng.integers(1, 4))      # whole chunks: the staged path
+        sizes[i] = 1536 * int(rng.integers(1, 4))     # whole chunks: the staged path
     wl = _ragged_workload("adamw", "bf16", "bf16", 8)
     wl.tensors = [TensorSpec(f"t{i}", (n,), "normal", 0.02) for i, n in enumerate(sizes)]
     _run_full_compare(wl, 2)

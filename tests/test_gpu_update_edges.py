@@ -24,7 +24,7 @@ import gpu_util as U
 pytestmark = pytest.mark.gpu
 
 DEV = "cuda"
-CHUNK = 512  # one staged chunk of the kernel: every block below fills one
+CHUNK = 1536  # whole staged chunks of the kernels (768 elements for AdamW with 8-bit ECC, 512 otherwise)
 
 
 @pytest.fixture(scope="module", autouse=True)
