@@ -100,19 +100,38 @@ struct StepLaunch {
     int64_t chunk;  // elements per chunk
 };
 
-template <int WDT, int GDT, int NB, int KIND>
+template <int WDT, int GDT, int NB, int KIND, bool WIDE>
 StepLaunch step_launch()
 {
-    using G = fo::Geometry<NB, KIND>;
-    return {fo::step_kernel<WDT, GDT, NB, KIND>, G::kBlockThreads, fo::step_smem_bytes<NB, KIND>(), G::kChunk};
+    using G = fo::Geometry<NB, KIND, WIDE>;
+    return {fo::step_kernel<WDT, GDT, NB, KIND, WIDE>, G::kBlockThreads, fo::step_smem_bytes<NB, KIND, WIDE>(),
+            G::kChunk};
+}
+
+// the geometry for a call over `total` elements: wide chunks for AdamW with
+// 8-bit ECC codes once the call is large enough
+template <int WDT, int GDT, int NB, int KIND>
+StepLaunch sized_launch(int64_t total)
+{
+    if constexpr (NB == 8 && fo::uses_v(KIND)) {
+        if (total >= fo::kWideMinElems) return step_launch<WDT, GDT, NB, KIND, true>();
+    }
+    return step_launch<WDT, GDT, NB, KIND, false>();
+}
+
+int64_t total_numel(const fo_tensor* t, int n)
+{
+    int64_t s = 0;
+    for (int i = 0; i < n; i++) s += t[i].numel;
+    return s;
 }
 
 // the step kernel of a format (k = nullptr if the format is not provided)
 template <int KIND>
-StepLaunch pick_step(const fo_format& f)
+StepLaunch pick_step(const fo_format& f, int64_t total)
 {
 #define FO_PICK(W, G, N)                                                                  \
-    if (f.w_dtype == W && f.grad_dtype == G && f.ecc_bits == N) return step_launch<W, G, N, KIND>();
+    if (f.w_dtype == W && f.grad_dtype == G && f.ecc_bits == N) return sized_launch<W, G, N, KIND>(total);
     FO_PICK(0, 0, 8) FO_PICK(0, 1, 8) FO_PICK(1, 0, 8) FO_PICK(1, 1, 8)
     FO_PICK(0, 0, 16) FO_PICK(0, 1, 16) FO_PICK(1, 0, 16) FO_PICK(1, 1, 16)
 #undef FO_PICK
@@ -283,7 +302,7 @@ fo_status fo_adamw_step(const fo_tensor* t, int n_tensors, fo_format f, const fo
     sc.s[6] = (float)h->eps;
     sc.s[7] = (float)(1.0 - h->lr * h->weight_decay);
     adamw_fast_bounds(sc);
-    const StepLaunch L = pick_step<fo::kAdamW>(f);
+    const StepLaunch L = pick_step<fo::kAdamW>(f, total_numel(t, n_tensors));
     if (!L.k) return fail(FO_ERR_UNSUPPORTED, "format not provided");
     return launch_step(L, sc, t, n_tensors, (cudaStream_t)stream);
 }
@@ -312,7 +331,7 @@ fo_status fo_sgdm_step(const fo_tensor* t, int n_tensors, fo_format f, const fo_
     sc.s[5] = h->step == 1 ? 1.0f : 0.0f;
     sc.s[6] = 0.0f;
     sc.s[7] = 0.0f;
-    const StepLaunch L = pick_step<fo::kSGDM>(f);
+    const StepLaunch L = pick_step<fo::kSGDM>(f, total_numel(t, n_tensors));
     if (!L.k) return fail(FO_ERR_UNSUPPORTED, "format not provided");
     return launch_step(L, sc, t, n_tensors, (cudaStream_t)stream);
 }
@@ -327,9 +346,12 @@ fo_status fo_stream_copy(const fo_tensor* t, int n_tensors, fo_format f, int ada
     if (n_tensors == 0) return FO_OK;
     fo::Scalars sc = {};
     // the copy moves bytes only: the 16-bit formats do not matter, the ECC width does
+    const int64_t total = total_numel(t, n_tensors);
     StepLaunch L;
-    if (adamw_mix) L = f.ecc_bits == 8 ? step_launch<0, 0, 8, fo::kCopyAdamW>() : step_launch<0, 0, 16, fo::kCopyAdamW>();
-    else L = f.ecc_bits == 8 ? step_launch<0, 0, 8, fo::kCopySGDM>() : step_launch<0, 0, 16, fo::kCopySGDM>();
+    if (adamw_mix)
+        L = f.ecc_bits == 8 ? sized_launch<0, 0, 8, fo::kCopyAdamW>(total) : sized_launch<0, 0, 16, fo::kCopyAdamW>(total);
+    else
+        L = f.ecc_bits == 8 ? sized_launch<0, 0, 8, fo::kCopySGDM>(total) : sized_launch<0, 0, 16, fo::kCopySGDM>(total);
     return launch_step(L, sc, t, n_tensors, (cudaStream_t)stream);
 }
 

@@ -54,6 +54,10 @@
  *   - numel == 0 tensors are skipped; n_tensors == 0 is a no-op.
  *   - Results do not depend on the number of tensors per call, their order,
  *     or on whether they are stepped in one call or one call per tensor.
+ *   - Launch geometry (performance only, results identical): AdamW calls with
+ *     8-bit ECC codes over at least 3 * 2^25 elements in total use chunks of 768
+ *     elements in 10-warp blocks, every other call chunks of 512 elements in
+ *     8-warp blocks; a tensor's last partial chunk takes the scalar path.
  */
 #ifndef FO_H
 #define FO_H

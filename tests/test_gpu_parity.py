@@ -120,12 +120,18 @@ def test_encode_decode_master_bit_exact(wdt, nbits):
 
 # ---- flat group, 10 steps, every byte ----------------------------------------------
 
-def _run_full_compare(wl, steps, order=None, check_every=True):
+def _run_full_compare(wl, steps, order=None, check_every=True, sample_above=None):
+    """Every byte of every tensor against the oracle; tensors of more than
+    `sample_above` elements on 256 sampled groups (first and last included)."""
     P = U.device_state(wl)
     G = U.GradArena(P)
     orcs = []
+    rng = np.random.default_rng(23)
     for ti, t in enumerate(wl.tensors):
-        orcs.append(U.OracleSample(wl, ti, np.arange((t.numel + 31) // 32), threads=_nthreads()))
+        ng = (t.numel + 31) // 32
+        sampled = sample_above is not None and t.numel > sample_above
+        groups = U.sample_groups(t.numel, 256, rng) if sampled else np.arange(ng)
+        orcs.append(U.OracleSample(wl, ti, groups, threads=_nthreads()))
     for t in range(1, steps + 1):
         G.fill(wl, t)
         U.step(wl, P, G, t, order=order)
@@ -164,6 +170,23 @@ def _ragged_workload(opt, wdt, gdt, nbits):
 def test_ragged_multitensor_all_formats(opt, wdt, gdt, nbits):
     wl = _ragged_workload(opt, wdt, gdt, nbits)
     _run_full_compare(wl, 3)
+
+
+# calls of AdamW with 8-bit ECC codes over at least 3 * 2^25 elements take
+# the wide launch geometry (chunks of 768 elements in 10-warp blocks)
+WIDE_MIN = 3 << 25
+
+
+@pytest.mark.parametrize("wdt,gdt", [("bf16", "bf16"), ("fp16", "fp16"), ("bf16", "fp16"), ("fp16", "bf16")])
+def test_ragged_wide_geometry(wdt, gdt):
+    """The ragged list plus one tensor of 3 * 2^25 + 45 elements: the call is
+    large enough for the wide geometry, so every tensor (ragged tails, chunk
+    edges at 767 / 768 / 769 and 1536 / 1537) goes through it; every byte of
+    every ragged tensor and sampled groups of the large one against the
+    oracle."""
+    wl = _ragged_workload("adamw", wdt, gdt, 8)
+    wl.tensors.insert(7, TensorSpec("fill", (WIDE_MIN + 45,), "normal", 0.02))
+    _run_full_compare(wl, 2, sample_above=1 << 20)
 
 
 @pytest.mark.parametrize("hp", [
@@ -247,17 +270,22 @@ def test_empty_and_tiny_tensors_in_one_call():
         assert all(v == 0 for v in U.mismatches(exp, U.gather_device(P, ti, exp)).values())
 
 
-def test_many_tensors_split_across_launches():
+@pytest.mark.parametrize("fill", [0, WIDE_MIN])
+def test_many_tensors_split_across_launches(fill):
     """1000 tensors in one call: more than one launch's parameter block holds
-    (384 descriptors), so the call is split into several launches.  Every
-    byte of every tensor against the oracle."""
+    (384 descriptors), so the call is split into several launches (with a
+    3 * 2^25-element tensor in the middle, all of them in the wide geometry).
+    Every byte of every tensor (sampled groups of the large one) against the
+    oracle."""
     rng = np.random.default_rng(17)
     sizes = [int(v) for v in rng.integers(1, 2600, 1000)]
     for i in range(0, 1000, 97):
         sizes[i] = 1536 * int(rng.integers(1, 4))     # whole chunks: the staged path
+    if fill:
+        sizes[500] = fill
     wl = _ragged_workload("adamw", "bf16", "bf16", 8)
     wl.tensors = [TensorSpec(f"t{i}", (n,), "normal", 0.02) for i, n in enumerate(sizes)]
-    _run_full_compare(wl, 2)
+    _run_full_compare(wl, 2, sample_above=1 << 20)
 
 
 # ---- gradient release == one multi-tensor launch -------------------------------------
