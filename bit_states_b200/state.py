@@ -2,8 +2,9 @@
 
 Buffers are allocated with torch (plumbing only) as one arena per stream of
 bytes: downcast weights, ECC codes, momentum codes + scales, variance codes +
-scales.  Each tensor's slice starts on a multiple of 512 elements, so every
-array of every tensor is aligned for the kernels' 256-bit accesses.  All
+scales.  Each tensor's slice starts on a multiple of 512 elements (its
+scales on a multiple of 16 groups), so every array of every tensor starts on
+a 16-byte boundary, as the kernels' staged path needs.  All
 arithmetic (encode, step, decode) runs in libfo's kernels.
 """
 from __future__ import annotations

@@ -171,8 +171,9 @@ __global__ void k_codec(unsigned long long* cnt, uint32_t* ex)
     const uint32_t lim = W == 0 ? 0x7F7F8000u : 0x477FF000u;  // kDecodeLimit, 65520
     for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (uint64_t)lim; i += stride) {
         const float xa = __uint_as_float((uint32_t)i), xb = -xa;
-        int c0, c1;
-        const uint32_t wo = fo::fast_encode_pair<W, 8>(make_float2(xa, xb), c0, c1);
+        uint32_t codes;
+        const uint32_t wo = fo::fast_encode_pair<W, 8>(make_float2(xa, xb), codes);
+        const int c0 = (int)(int16_t)(codes & 0xFFFFu), c1 = (int)(int16_t)(codes >> 16);
         const uint32_t pa = fo::downcast16<W>(xa), pb = fo::downcast16<W>(xb);
         if ((wo & 0xFFFFu) != pa || (wo >> 16) != pb || c0 != fo::ecc_encode<W, 8>(xa, pa) ||
             c1 != fo::ecc_encode<W, 8>(xb, pb))
