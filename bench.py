@@ -194,7 +194,10 @@ def cpu_sample(wl, n_params: int, rank_seed: int = 0):
     return w, e, gb
 
 
-def time_oracle(wl, n_params: int, steps: int, warmup: int, threads: int):
+def time_oracle(wl, n_params: int, steps: int, warmup: int, threads: int, min_seconds: float = 0.0):
+    """Oracle throughput on a bounded sample: `warmup` untimed steps, then
+    `steps` timed steps, continued until at least `min_seconds` have passed.
+    Returns (Gparams/s, seconds, params per step, timed steps)."""
     import oracle
 
     w, e, gb = cpu_sample(wl, n_params)
@@ -215,11 +218,13 @@ def time_oracle(wl, n_params: int, steps: int, warmup: int, threads: int):
     for t in range(1, warmup + 1):
         one(t)
     t0 = time.perf_counter()
-    for k in range(steps):
+    k = 0
+    while k < steps or time.perf_counter() - t0 < min_seconds:
         one(warmup + 1 + k)
+        k += 1
     dt = time.perf_counter() - t0
     n = w.size
-    return n * steps / dt / 1e9, dt, n
+    return n * k / dt / 1e9, dt, n, k
 
 
 def arm_config(wl, args, world):
@@ -244,8 +249,8 @@ def run_reference(args, rank, world):
     # each step is a bounded sample of the workload sized to keep the whole
     # run within a few minutes of host time
     n_params = min(args.cpu_sample_params, 1 << 24)
-    value, dt, n = time_oracle(wl, n_params, args.steps if args.steps <= 20 else 20, min(args.warmup, 3), threads)
-    steps = args.steps if args.steps <= 20 else 20
+    value, dt, n, steps = time_oracle(wl, n_params, args.steps if args.steps <= 20 else 20, min(args.warmup, 3),
+                                      threads)
     sample = f"{n} params per step (whole 32-groups drawn from all {len(wl.tensors)} tensors of {wl.name}), " \
              f"AdamW step 1.., {threads} host threads"
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "Gparams/s",
@@ -431,10 +436,11 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         threads = os.cpu_count() or 1
-        v, dt, n = time_oracle(wl, args.cpu_sample_params, 1, 1, threads)
+        v, dt, n, k = time_oracle(wl, args.cpu_sample_params, 1, 1, threads, min_seconds=10.0)
         cpu = {"value": round(v, 6), "unit": "Gparams/s", "cores": threads, "kind": "oracle",
-               "sample": f"{n} params (whole 32-groups drawn from all {len(wl.tensors)} tensors), one "
-                         f"{wl.optimizer} step after one warm step, {threads} host threads, {dt:.2f} s"}
+               "sample": f"{n} params (whole 32-groups drawn from all {len(wl.tensors)} tensors), "
+                         f"{k} {wl.optimizer} steps after one warm step, {threads} host threads, "
+                         f"{dt:.2f} s timed"}
 
     if rank == 0:
         line = {
