@@ -160,10 +160,14 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower().startswith("active")})
         pload = [p for p in pw if p > 200.0] or pw
+        # nvidia-smi's power reading trails the load (it averages over a window),
+        # so the steady figure is the median of the second half of the samples
+        steady = pload[len(pload) // 2:]
         return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": max(mx) if mx else None,
                 "reasons": reasons, "samples": len(rows), "samples_under_load": len(load),
                 "power_w_max": max(pw) if pw else None,
-                "power_w_median": statistics.median(pload) if pload else None}
+                "power_w_median": statistics.median(pload) if pload else None,
+                "power_w_steady": statistics.median(steady) if steady else None}
 
 
 # ---------------------------------------------------------------------------
@@ -400,7 +404,7 @@ def main():
 
         for _ in range(3):
             do_copy()
-        Kc = min(K, 50)
+        Kc = K  # as many launches as the timed steps, so that clocks and power settle alike
         cs = [torch.cuda.Event(enable_timing=True) for _ in range(Kc)]
         ce = [torch.cuda.Event(enable_timing=True) for _ in range(Kc)]
         csampler = ClockSampler(gpu_id)
@@ -419,6 +423,39 @@ def main():
             tc = torch.tensor([ceiling_ms], dtype=torch.float64, device=dev)
             dist.all_reduce(tc, op=dist.ReduceOp.MAX)
             ceiling_ms = float(tc[0])
+
+    # ---- a plain two-stream device copy (torch) for the same time: the HBM
+    # reference point for the power the byte mix itself draws ----
+    plain = None
+    if args.launch_mode == "multi" and ceiling_ms is not None:
+        nb = 4 << 30
+        src = torch.empty(nb, dtype=torch.uint8, device=dev)
+        dst = torch.empty(nb, dtype=torch.uint8, device=dev)
+        src.fill_(1)
+        for _ in range(3):
+            dst.copy_(src)
+        torch.cuda.synchronize()
+        one = torch.cuda.Event(enable_timing=True)
+        two = torch.cuda.Event(enable_timing=True)
+        one.record(stream)
+        dst.copy_(src)
+        two.record(stream)
+        torch.cuda.synchronize()
+        Kp = max(10, int(ceiling_ms * Kc / max(one.elapsed_time(two), 1e-3)))
+        psampler = ClockSampler(gpu_id)
+        psampler.start()
+        torch.cuda.synchronize()
+        one.record(stream)
+        for _ in range(Kp):
+            dst.copy_(src)
+        two.record(stream)
+        torch.cuda.synchronize()
+        pclocks = psampler.stop()
+        pms = one.elapsed_time(two) / Kp
+        plain = {"kernel": "torch copy_ of a 4 GiB buffer (one read and one write stream)",
+                 "achieved": round(2 * nb / (pms / 1e3) / 1e9, 1), "unit": "GB/s", "launches": Kp,
+                 "clocks": {k: pclocks.get(k) for k in ("sm_mhz", "power_w_median", "power_w_steady")}}
+        del src, dst
 
     n_params = wl.numel
     value = world * n_params * K / (total_ms / 1e3) / 1e9
@@ -458,7 +495,9 @@ def main():
                 "achieved": round(abytes / (ceiling_ms / 1e3) / 1e9, 1), "unit": "GB/s",
                 "frac_of_peak": round(abytes / (ceiling_ms / 1e3) / 1e9 / peak, 4),
                 "step_frac_of_ceiling": round(ceiling_ms / per_launch_ms, 4),
-                "clocks": {k: ceiling_clocks.get(k) for k in ("sm_mhz", "power_w_median", "power_w_max")}},
+                "clocks": {k: ceiling_clocks.get(k) for k in ("sm_mhz", "power_w_median", "power_w_steady",
+                                                              "power_w_max")},
+                "plain_copy": plain},
             "clocks": clocks,
             "gpu_launches": K * launches_per_step,
             "e2e": e2e,

@@ -89,9 +89,9 @@ typedef enum { FO_DT_BF16 = 0, FO_DT_FP16 = 1 } fo_dtype;
    one launch's parameter block are split into several launches. */
 #define FO_MAX_TENSORS_PER_CALL (1 << 20)
 
-/* Largest numel of one tensor (2^40 elements; larger ones are rejected with
-   FO_ERR_INVALID_ARG). */
-#define FO_MAX_NUMEL ((int64_t)1 << 40)
+/* Largest numel of one tensor (2^36 elements, far beyond what one GPU's
+   memory holds; larger ones are rejected with FO_ERR_INVALID_ARG). */
+#define FO_MAX_NUMEL ((int64_t)1 << 36)
 
 /* One parameter tensor.  All pointers are device memory owned by the caller.
    Optimizer fields that a call does not use may be NULL (v_q / v_scale for
