@@ -144,17 +144,30 @@ def _adamw_step_fn(fmt, hp):
     return step
 
 
+def _sgdm_step_fn(fmt, hp):
+    from . import fo
+
+    def step(state, grad, t, stream):
+        h = fo.fo_sgdm_hparams(hp["lr"], hp["momentum"], hp.get("dampening", 0.0), hp.get("weight_decay", 0.0),
+                               int(bool(hp.get("nesterov", False))), t)
+        fo.fo_sgdm_step(fo.descriptors([state], [grad]), 1, fmt, h, stream)
+
+    return step
+
+
 class DataParallelStep:
     """Reduce-scatter -> fused step on the owned groups -> all-gather of x',
     bucket by bucket.
 
     ``step_fn(state, grad_shard, t, stream)`` steps one bucket slice in place
-    (default: the library's fused AdamW).  ``reduce_op`` is "sum" or "avg"
-    (the average needs a backend that provides it, such as NCCL)."""
+    (default: the library's fused step for ``optimizer``, "adamw" or "sgdm",
+    with ``hparams``; SGD-momentum needs a state built with ``adam=False``).
+    ``reduce_op`` is "sum" or "avg" (the average needs a backend that
+    provides it, such as NCCL)."""
 
     def __init__(self, state: ShardedState, group=None, step_fn: Optional[Callable] = None,
                  fmt=None, hparams=None, reduce_op: str = "sum", grad_dtype: str = "bf16",
-                 w_dtype: str = "bf16"):
+                 w_dtype: str = "bf16", optimizer: str = "adamw"):
         import torch
         import torch.distributed as dist
 
@@ -165,10 +178,15 @@ class DataParallelStep:
         self.gdt, self.wdt = tdt[grad_dtype], tdt[w_dtype]
         self.group = group
         self.layout = state.layout
+        if optimizer not in ("adamw", "sgdm"):
+            raise ValueError("optimizer must be 'adamw' or 'sgdm'")
+        if (optimizer == "adamw") != state.adam:
+            raise ValueError("the state's variance arrays do not match the optimizer")
         if step_fn is None:
             from . import fo
 
-            step_fn = _adamw_step_fn(fmt or fo.make_format(), hparams)
+            fmt = fmt or fo.make_format(w_dtype, grad_dtype, state.ecc_bits)
+            step_fn = (_adamw_step_fn if optimizer == "adamw" else _sgdm_step_fn)(fmt, hparams)
         self.step_fn = step_fn
         self.op = {"sum": dist.ReduceOp.SUM, "avg": dist.ReduceOp.AVG}[reduce_op]
         dev = state.w.device

@@ -153,3 +153,126 @@ def test_two_rank_dp_step_equals_single_process():
                 assert np.array_equal(mq[k * GROUP:k * GROUP + L], exp[ti].mq[a:b]), (rank, ti, lg)
                 assert np.array_equal(vq[k * GROUP:k * GROUP + L], exp[ti].vq[a:b]), (rank, ti, lg)
                 assert ms.view(np.uint16)[k] == exp[ti].ms[lg] and vs.view(np.uint16)[k] == exp[ti].vs[lg]
+
+
+# ---- SGD-momentum, fp16 weights and gradients, three ranks ---------------------------
+
+SGD_HP = dict(lr=0.1, momentum=0.9, dampening=0.0, weight_decay=1e-4, nesterov=False)
+
+
+def _small_int_grads(rank, ti, t, n):
+    """fp16 gradients k * 2^-12 with small integers k in [-8, 8]: the sum over
+    three ranks is exact in fp16 in every order, so the collective's
+    reduction order cannot change the reference."""
+    from workloads import gen
+
+    u = gen.normal(gen.stream_key(rank + 11, ti, t, gen.KIND_GRAD), np.arange(n), 1.0)
+    k = np.clip(np.rint(3.0 * u), -8, 8).astype(np.int32)
+    return k
+
+
+def _to_fp16_bits(k):
+    return (k.astype(np.float32) * np.float32(2.0 ** -12)).astype(np.float16).view(np.uint16)
+
+
+def _oracle_sgdm_step_fn(state, grad, t, stream):
+    import oracle
+
+    st = oracle.State(state.w.numpy().view(np.uint16), state.ecc.numpy(), state.m_q.numpy(),
+                      state.m_scale.numpy().view(np.uint16))
+    oracle.sgdm_step(st, grad.numpy().view(np.uint16), **SGD_HP, step=t, wdt=oracle.FP16, gdt=oracle.FP16)
+
+
+def _sgd_worker(rank, world, port, q):
+    import torch
+    import torch.distributed as dist
+
+    import oracle
+    from bit_states_b200.dp import DataParallelStep, ShardedState
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        layout = FlatLayout(NUMELS, world, bucket_groups=BUCKET_GROUPS)
+        st = ShardedState(layout, rank, "cpu", adam=False)
+        w, e = zip(*[oracle.encode_master(_masters(ti, n), oracle.FP16) for ti, n in enumerate(NUMELS)])
+        wf, ef = _flat(layout, w, np.uint16), _flat(layout, e, np.int8)
+        st.w.copy_(torch.from_numpy(wf.view(np.int16)))
+        for s0, s1, go in st.slices:
+            st.ecc[go * GROUP:go * GROUP + (s1 - s0)] = torch.from_numpy(ef[s0:s1])
+        dp = DataParallelStep(st, step_fn=_oracle_sgdm_step_fn, reduce_op="sum", grad_dtype="fp16",
+                              w_dtype="fp16", optimizer="sgdm")
+        for t in (1, 2, 3):
+            g = _flat(layout, [_to_fp16_bits(_small_int_grads(rank, ti, t, n)) for ti, n in enumerate(NUMELS)],
+                      np.uint16)
+            dp.step(torch.from_numpy(g.view(np.int16)), t)
+        q.put((rank, st.w.numpy().copy(), st.ecc.numpy().copy(), st.m_q.numpy().copy(),
+               st.m_scale.numpy().copy(), list(st.slices)))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_three_rank_sgdm_fp16_equals_single_process():
+    import oracle
+
+    world = 3
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_sgd_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = {}
+    for _ in range(world):
+        r = q.get(timeout=300)
+        res[r[0]] = r[1:]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    layout = FlatLayout(NUMELS, world, bucket_groups=BUCKET_GROUPS)
+    exp = []
+    for ti, n in enumerate(NUMELS):
+        w, e = oracle.encode_master(_masters(ti, n), oracle.FP16)
+        st = oracle.State.zeros_like_master(w, e, adam=False)
+        for t in (1, 2, 3):
+            ksum = sum(_small_int_grads(r, ti, t, n) for r in range(world))
+            oracle.sgdm_step(st, _to_fp16_bits(ksum), **SGD_HP, step=t, wdt=oracle.FP16, gdt=oracle.FP16)
+        exp.append(st)
+    seen = 0
+    for rank in range(world):
+        w, ecc, mq, ms, slices = res[rank]
+        for ti, n in enumerate(NUMELS):
+            o = layout.offsets[ti]
+            assert np.array_equal(w[o:o + n].view(np.uint16), exp[ti].w), (rank, ti)
+        for s0, s1, go in slices:
+            for g in range(s0 // GROUP, s1 // GROUP):
+                e0 = g * GROUP
+                ti = max(i for i in range(len(NUMELS)) if layout.offsets[i] <= e0)
+                lg = (e0 - layout.offsets[ti]) // GROUP
+                n = NUMELS[ti]
+                if lg * GROUP >= n:
+                    continue
+                k = go + (g - s0 // GROUP)
+                a, b = lg * GROUP, min(n, lg * GROUP + GROUP)
+                L = b - a
+                assert np.array_equal(ecc[k * GROUP:k * GROUP + L], exp[ti].ecc[a:b]), (rank, ti, lg)
+                assert np.array_equal(mq[k * GROUP:k * GROUP + L], exp[ti].mq[a:b]), (rank, ti, lg)
+                assert ms.view(np.uint16)[k] == exp[ti].ms[lg]
+                seen += 1
+    assert seen == sum((n + 31) // 32 for n in NUMELS)   # every real group owned by exactly one rank
+
+
+def test_dp_step_rejects_mismatched_optimizer():
+    import pytest
+
+    from bit_states_b200.dp import DataParallelStep, ShardedState
+
+    layout = FlatLayout(NUMELS, 1, bucket_groups=BUCKET_GROUPS)
+    with pytest.raises(ValueError):
+        DataParallelStep(ShardedState(layout, 0, "cpu", adam=True), step_fn=lambda *a: None, optimizer="sgdm")
+    with pytest.raises(ValueError):
+        DataParallelStep(ShardedState(layout, 0, "cpu", adam=False), step_fn=lambda *a: None)
+    with pytest.raises(ValueError):
+        DataParallelStep(ShardedState(layout, 0, "cpu"), step_fn=lambda *a: None, optimizer="lamb")
