@@ -276,3 +276,39 @@ def test_dp_step_rejects_mismatched_optimizer():
         DataParallelStep(ShardedState(layout, 0, "cpu", adam=False), step_fn=lambda *a: None)
     with pytest.raises(ValueError):
         DataParallelStep(ShardedState(layout, 0, "cpu"), step_fn=lambda *a: None, optimizer="lamb")
+
+
+def test_layout_properties_random_lists():
+    """Property test of the flat layout: for random parameter lists, world
+    sizes and bucket sizes, every tensor starts on a group boundary and its
+    groups lie inside the layout, buckets tile the groups in order with sizes
+    that are multiples of the world size, and every rank's slices are equal,
+    disjoint and together cover every group exactly once."""
+    from hypothesis import given, settings
+    from hypothesis import strategies as hs
+
+    @settings(max_examples=200, deadline=None)
+    @given(hs.lists(hs.integers(0, 5000), min_size=1, max_size=12), hs.integers(1, 8), hs.integers(1, 300))
+    def check(numels, world, bucket_groups):
+        L = FlatLayout(numels, world, bucket_groups=bucket_groups)
+        off = 0
+        for o, n in zip(L.offsets, numels):
+            assert o % GROUP == 0 and o == off
+            off += (n + GROUP - 1) // GROUP * GROUP
+        assert off <= L.numel == L.groups * GROUP
+        g = 0
+        for b in L.buckets:
+            assert b.g0 == g and b.groups > 0 and b.groups % world == 0
+            g += b.groups
+        assert g == L.groups
+        owned = np.zeros(L.groups, np.int32)
+        for r in range(world):
+            for b in L.buckets:
+                g0, k = b.shard(world, r)
+                assert k == b.groups // world and b.g0 <= g0 and g0 + k <= b.g0 + b.groups
+                owned[g0:g0 + k] += 1
+        assert np.all(owned == 1)
+        # only the last bucket is rounded up to a multiple of the world size
+        assert 0 <= L.groups - off // GROUP < world
+
+    check()
