@@ -99,3 +99,48 @@ def test_two_rank_shards_equal_whole_list():
         assert np.array_equal(cat(0), st.w) and np.array_equal(cat(1), st.ecc)
         assert np.array_equal(cat(2), st.mq) and np.array_equal(cat(3), st.ms)
         assert np.array_equal(cat(4), st.vq) and np.array_equal(cat(5), st.vs)
+
+
+def test_spans_properties_random_lists():
+    """Property test of the partition: for random lists and world sizes every
+    group is owned by exactly one rank, ranks own contiguous runs in list order
+    with sizes differing by at most one group, and the sliced views of
+    shard_states cover each span's elements and scales exactly."""
+    import torch
+    from hypothesis import given, settings
+    from hypothesis import strategies as hs
+
+    from bit_states_b200.fo import TensorState
+    from bit_states_b200.shard import shard_states
+
+    @settings(max_examples=200, deadline=None)
+    @given(hs.lists(hs.integers(0, 3000), min_size=1, max_size=10), hs.integers(1, 9))
+    def check(numels, world):
+        flat_owner = []
+        for r in range(world):
+            spans = shard_spans(numels, world, r)
+            for sp in spans:
+                assert 0 <= sp.g0 < sp.g1 <= (sp.numel + GROUP - 1) // GROUP
+                flat_owner.extend([(sp.tensor, g, r) for g in range(sp.g0, sp.g1)])
+            states = [TensorState(torch.zeros(n, dtype=torch.int16), torch.zeros(n, dtype=torch.int8),
+                                  torch.zeros(n, dtype=torch.int8), torch.zeros((n + 31) // 32, dtype=torch.int16),
+                                  torch.zeros(n, dtype=torch.uint8), torch.zeros((n + 31) // 32, dtype=torch.int16))
+                      for n in numels]
+            grads = [torch.zeros(n, dtype=torch.int16) for n in numels]
+            ss, gg = shard_states(states, grads, spans)
+            for sp, st, g in zip(spans, ss, gg):
+                assert st.w.numel() == st.ecc.numel() == st.m_q.numel() == st.v_q.numel() == g.numel() == sp.elems
+                assert st.m_scale.numel() == st.v_scale.numel() == sp.g1 - sp.g0
+                # the views start where the span starts (storage offsets, in elements)
+                assert st.w.storage_offset() == sp.e0 and st.m_scale.storage_offset() == sp.g0
+        # in list order: (tensor, group) keys ascending, owners non-decreasing
+        keys = sorted(flat_owner)
+        assert keys == sorted(set(keys))                  # each group once
+        assert [(t, g) for t, g, _ in keys] == [(ti, g) for ti, n in enumerate(numels)
+                                                for g in range((n + 31) // 32)]
+        owners = [r for _, _, r in keys]
+        assert owners == sorted(owners)
+        sizes = [owners.count(r) for r in range(world)]
+        assert max(sizes) - min(sizes) <= 1
+
+    check()
