@@ -49,7 +49,12 @@
  *      root, bias correction), on the decoded f32 state; SGD-momentum as in
  *      torch.optim.SGD (coupled decay, dampening, optional Nesterov,
  *      first step copies the gradient into the buffer).
- *   R9 NaN codes: a NaN value quantizes to code 0.
+ *   R9 non-finite values: a NaN downcasts to the positive quiet NaN of the
+ *      format (bf16 0x7FC0, fp16 0x7E00) whatever its sign and payload, with
+ *      ECC 0 (as every non-finite x'); inf and NaN state values are left out
+ *      of the group maximum and get code 0; everything else follows IEEE
+ *      binary32 arithmetic (an inf gradient gives m' = inf, v' = inf and, in
+ *      AdamW, the quotient inf/inf = NaN).
  *
  * Parity pins (tests/test_oracle_*.py): the downcast against numpy and torch
  * casts over all 2^32 binary32 patterns; the ECC against closed integer
@@ -127,12 +132,15 @@ static uint16_t fmt_pattern_exact(fmt_t f, double r)
     return (uint16_t)(((unsigned)(E + f.bias) << (f.p - 1)) | (unsigned)m);
 }
 
-/* R1: round-to-nearest-even downcast of a binary32 value */
+/* R1: round-to-nearest-even downcast of a binary32 value.  R9: every NaN,
+   whatever its sign and payload, becomes the one positive quiet NaN of the
+   format (only the quiet bit set): a NaN carries no sign or payload that
+   binary32 arithmetic on different machines would agree on. */
 static uint16_t fmt_round_rne(fmt_t f, float xf)
 {
     double x = xf;
     uint16_t sign = signbit(x) ? 0x8000 : 0;
-    if (isnan(x)) return (uint16_t)(sign | fmt_qnan_bits(f));
+    if (isnan(x)) return fmt_qnan_bits(f);
     double a = fabs(x);
     if (isinf(a)) return (uint16_t)(sign | fmt_inf_bits(f));
     if (a == 0.0) return sign;
@@ -231,10 +239,16 @@ static float ecc_decode(fmt_t f, int nbits, uint16_t xp_bits, int32_t rho)
 
 #define GROUP 32
 
+/* R9: a non-finite state value (inf or NaN) has no place on a scaled 8-bit
+   grid; it is left out of its group's maximum and stored as code 0, so that
+   one overflowed element does not flatten the codes of the other 31. */
+static int finite_f(float z) { return isfinite(z) != 0; }
+
 static float group_absmax(const float* z, int n)
 {
     float A = 0.0f;
-    for (int i = 0; i < n; i++) A = fmaxf(A, fabsf(z[i]));
+    for (int i = 0; i < n; i++)
+        if (finite_f(z[i])) A = fmaxf(A, fabsf(z[i]));
     return A;
 }
 
@@ -250,6 +264,10 @@ static void m_encode_group(const float* z, int n, int8_t* q, uint16_t* S_bits)
     }
     float r = 1.0f / Sf;
     for (int i = 0; i < n; i++) {
+        if (!finite_f(z[i])) {
+            q[i] = 0;
+            continue;
+        }
         float y = z[i] * r;
         float num = 2.0f * y;
         float den = 1.0f + fabsf(y);
@@ -283,6 +301,10 @@ static void v_encode_group(const float* sv, int n, uint8_t* q, uint16_t* S_bits)
     }
     float k = 255.0f / Sf;
     for (int i = 0; i < n; i++) {
+        if (!finite_f(sv[i])) {
+            q[i] = 0;
+            continue;
+        }
         float t = sv[i] * k;
         float c = nearbyintf(t);
         if (isnan(c) || c < 0.0f) c = 0.0f;
@@ -663,7 +685,7 @@ int oracle_quantize_fixed_scale(const float* z, void* q, uint16_t S, int64_t n, 
     float Sf = (float)fmt_value(F_FP16, S);
     for (int64_t i = 0; i < n; i++) {
         float k;
-        if (Sf == 0.0f) {
+        if (Sf == 0.0f || !finite_f(z[i])) {
             k = 0.0f;
         } else if (kind == 0) {
             float r = 1.0f / Sf;

@@ -35,9 +35,11 @@ def _compare(orc, pats: np.ndarray, wdt: int):
     got = orc.downcast(x, wdt, threads=threads())
     exp = _lib_bf16(x) if wdt == BF16 else _lib_fp16(x)
     nan = np.isnan(x)
-    # NaN: only NaN-ness and sign are specified
+    # NaN: the libraries disagree on sign and payload (torch's bf16 cast gives
+    # 0xFFFF, torch's fp16 cast and numpy keep sign and payload bits); the
+    # reading fixes one positive quiet NaN with only the quiet bit set
     assert np.all(_is_nan_bits(got[nan], wdt))
-    assert np.array_equal(got[nan] >> 15, (pats[nan] >> 31).astype(np.uint16))
+    assert np.all(got[nan] == (0x7FC0 if wdt == BF16 else 0x7E00))
     bad = np.nonzero(got[~nan] != exp[~nan])[0]
     assert bad.size == 0, f"{bad.size} mismatches, first x={x[~nan][bad[:4]]}"
 

@@ -14,6 +14,7 @@ import oracle
 from oracle.build import SRC, build
 
 import test_oracle_ecc as T_ecc
+import test_oracle_nonfinite as T_nf
 import test_oracle_states as T_st
 import test_oracle_update as T_up
 
@@ -36,9 +37,15 @@ MUTATIONS = [
      lambda o: T_st.test_momentum_compander_is_scaled_softsign(o)),
     ("scale rounded to nearest", "double k = ceil(a / ulp);", "double k = nearbyint(a / ulp);",
      lambda o: T_st.test_scale_is_fp16_round_up(o)),
-    ("variance code without the sqrt domain", "float k = 255.0f / Sf;\n    for (int i = 0; i < n; i++) {\n        float t = sv[i] * k;",
-     "float k = 255.0f / Sf;\n    for (int i = 0; i < n; i++) {\n        float t = sv[i] * sv[i] * k;",
+    ("variance code without the sqrt domain", "        float t = sv[i] * k;",
+     "        float t = sv[i] * sv[i] * k;",
      lambda o: T_st.test_variance_compander_is_sqrt(o)),
+    ("inf kept in the group maximum", "        if (finite_f(z[i])) A = fmaxf(A, fabsf(z[i]));",
+     "        if (!isnan(z[i])) A = fmaxf(A, fabsf(z[i]));",
+     lambda o: T_nf.test_nonfinite_state_values_stay_out_of_the_scale(o, 0)),
+    ("NaN downcast keeps its sign", "    if (isnan(x)) return fmt_qnan_bits(f);",
+     "    if (isnan(x)) return (uint16_t)(sign | fmt_qnan_bits(f));",
+     lambda o: T_nf.test_adamw_nonfinite_gradient_poisons_only_its_element(o, 0, 0, 8)),
     ("SGD weight decay with the wrong sign", "float g1 = fmaf(J->wd, x, gr);", "float g1 = fmaf(-J->wd, x, gr);",
      lambda o: T_up.test_sgdm_matches_torch(o, 0.0, False)),
 ]
