@@ -251,7 +251,8 @@ extern "C" {
 // |x (1-lr wd)| for which an update of at most
 //   U = |lr/(1-b1^t)| (2^-119 / eps + 2^-126)
 // cannot change x'' (U < |x (1-lr wd)| 2^-26), s[10] = the largest sqrt(v')
-// that keeps the divisor sqrt(v') / sqrt(1-b2^t) + eps at or below 2^20.
+// that keeps the divisor sqrt(v') / sqrt(1-b2^t) + eps at or below 2^20 and
+// the variance scale below its saturation at 65504 (the largest fp16).
 // Where those conditions cannot hold (eps < 2^-60, a step size too small to
 // scale by 2^-40) s[9] is +inf and every slice takes the exact path.
 static void adamw_fast_bounds(fo::Scalars& sc)
@@ -271,7 +272,7 @@ static void adamw_fast_bounds(fo::Scalars& sc)
     if ((double)t < thr) t = std::nextafter(t, inf);
     sc.s[9] = t;
     float b = (float)((std::ldexp(1.0, 20) - (double)eps) / (double)ibc2 * (1.0 - std::ldexp(1.0, -20)));
-    sc.s[10] = b;
+    sc.s[10] = b < 65504.0f ? b : 65504.0f;
 }
 
 fo_status fo_adamw_step(const fo_tensor* t, int n_tensors, fo_format f, const fo_adamw_hparams* h,

@@ -49,10 +49,13 @@ __device__ __forceinline__ float widen16(uint32_t h)
     }
 }
 
-// round to nearest even (overflow -> inf, NaN -> a quiet NaN)
+// round to nearest even (overflow -> inf); every NaN, whatever its sign and
+// payload, becomes the positive quiet NaN with only the quiet bit set (bf16
+// 0x7FC0, fp16 0x7E00): binary32 arithmetic gives NaNs no portable sign
 template <int DT>
 __device__ __forceinline__ uint32_t downcast16(float x)
 {
+    if (x != x) return DT == kBF16 ? 0x7FC0u : 0x7E00u;
     if constexpr (DT == kBF16) {
         return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x));
     } else {
@@ -145,9 +148,14 @@ __device__ __forceinline__ uint32_t scale_fp16_up(float a)
     return s > 0x7BFFu ? 0x7BFFu : s;
 }
 
+// a state value that takes part in its group's scale and gets a code: inf
+// and NaN do not (they are stored as code 0)
+__device__ __forceinline__ bool finite32(float z) { return fabsf(z) <= 3.40282347e38f; }
+
 // momentum: code = clamp(rint(127 * (2y / (1 + |y|))), +-127), y = z * r
 __device__ __forceinline__ int m_code(float z, float r)
 {
+    if (!finite32(z)) return 0;
     const float y = __fmul_rn(z, r);
     const float c = __fdiv_rn(__fmul_rn(2.0f, y), __fadd_rn(1.0f, fabsf(y)));
     int q = __float2int_rn(__fmul_rn(127.0f, c));
@@ -159,6 +167,7 @@ __device__ __forceinline__ int m_code(float z, float r)
 // variance: code = min(255, rint(sqrt(v) * k)), k = 255 / S
 __device__ __forceinline__ int v_code(float sv, float k)
 {
+    if (!finite32(sv)) return 0;
     int q = __float2int_rn(__fmul_rn(sv, k));
     q = q > 255 ? 255 : q;
     q = q < 0 ? 0 : q;

@@ -31,6 +31,13 @@
  *   grad     numel 16-bit gradients (bf16 or fp16), read only; gradients stay
  *            in backward precision.
  *
+ * Non-finite values (the pages are silent; a fixed reading): a NaN master
+ * is stored as the positive quiet NaN of its format (bf16 0x7FC0, fp16
+ * 0x7E00) with code 0, an inf master as inf with code 0; inf and NaN values
+ * of m' or sqrt(v') are left out of their group's maximum and stored as code
+ * 0; all other arithmetic is IEEE binary32 (an inf gradient makes the AdamW
+ * update inf / inf = NaN).
+ *
  * Conventions for every call:
  *   - Memory: the caller owns every buffer; the library allocates nothing and
  *     keeps no state between calls other than per-device launch constants
@@ -132,6 +139,12 @@ typedef struct {
 
 /*
  * fo_adamw_step - one fused AdamW step over n_tensors tensors.
+ * Passage: "FlashOptim: Breaking the Memory Wall with 24-bit Weights and
+ * Companded States" (wispaper blog), "Methodology" sections 1 (ULP-based
+ * weight splitting) and 2 (companded quantization) and "Performance" (one
+ * fused step); Davis Blalock's release thread, posts on the weight split,
+ * on 8-bit states with a 16-bit scale per 32 elements, on companding and on
+ * gradients kept in backward precision.
  * Per element: reconstruct x from (w, ecc); dequantize m and v with the
  * group scales; m' = b1*m + (1-b1)*g, v' = b2*v + (1-b2)*g^2 in binary32;
  * x'' = x*(1 - lr*wd) - lr/(1-b1^t) * m' / (sqrt(v')/sqrt(1-b2^t) + eps);
@@ -151,6 +164,9 @@ FO_API fo_status fo_adamw_step(const fo_tensor* t, int n_tensors, fo_format f,
  * momentum codes and scales only; v_q / v_scale are ignored).  Same format
  * support and error behaviour as fo_adamw_step; momentum and dampening must
  * lie in [0, 1].
+ * Passage: Davis Blalock's release thread, the post listing the optimizers
+ * the method wraps (Adam, SGD, ...), with the same weight split and momentum
+ * compander as fo_adamw_step.
  */
 FO_API fo_status fo_sgdm_step(const fo_tensor* t, int n_tensors, fo_format f,
                        const fo_sgdm_hparams* h, void* stream);
@@ -164,6 +180,7 @@ FO_API fo_status fo_sgdm_step(const fo_tensor* t, int n_tensors, fo_format f,
  * ceiling for the step on the same tensors.  Arguments, validation and errors
  * as fo_adamw_step / fo_sgdm_step; the 16-bit formats in f are not used, the
  * ECC width is.  Concurrent calls or steps on the same tensors race.
+ * Passage: none (a measurement aid, not part of the method).
  */
 FO_API fo_status fo_stream_copy(const fo_tensor* t, int n_tensors, fo_format f, int adamw_mix,
                         void* stream);
@@ -175,6 +192,9 @@ FO_API fo_status fo_stream_copy(const fo_tensor* t, int n_tensors, fo_format f, 
  * Errors: FO_ERR_INVALID_ARG (NULL pointer with n > 0, n < 0),
  * FO_ERR_UNSUPPORTED, FO_ERR_ALIGNMENT (x32 not 4-byte aligned, w or int16
  * ecc not 2-byte aligned), FO_ERR_CUDA.
+ * Passage: the wispaper blog's "1. ULP-based Weight Splitting"; the release
+ * thread's posts on the f32 interval that rounds to one downcast value and on
+ * integer-quantizing the position inside it.
  */
 FO_API fo_status fo_encode_master(const float* x32, void* w, void* ecc, int64_t n, fo_format f,
                            void* stream);
@@ -183,18 +203,20 @@ FO_API fo_status fo_encode_master(const float* x32, void* w, void* ecc, int64_t 
  * fo_decode_master - reconstruct n binary32 masters x32 (device) from w and
  * ecc (device).  Used to export checkpoints.  Same errors as
  * fo_encode_master.  Non-finite x' decode to x' itself.
+ * Passage: as fo_encode_master (the inverse of the split).
  */
 FO_API fo_status fo_decode_master(const void* w, const void* ecc, float* x32, int64_t n, fo_format f,
                            void* stream);
 
-/* Static English name of a status code. */
+/* Static English name of a status code.  Passage: none (error reporting). */
 FO_API const char* fo_status_string(fo_status s);
 
 /* Detail of the last non-FO_OK status returned on the calling thread
-   ("" if none).  The pointer stays valid until the next call on the thread. */
+   ("" if none).  The pointer stays valid until the next call on the thread.
+   Passage: none (error reporting). */
 FO_API const char* fo_last_error(void);
 
-/* Library version as major * 10000 + minor * 100 + patch. */
+/* Library version as major * 10000 + minor * 100 + patch.  Passage: none. */
 FO_API int fo_version(void);
 
 #ifdef __cplusplus

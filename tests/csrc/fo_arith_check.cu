@@ -181,6 +181,56 @@ __global__ void k_codec(unsigned long long* cnt, uint32_t* ex)
     }
 }
 
+// cnt[0]: div2_nr(x, b) != div.rn(x, b) over every pair of significands:
+// x in [1, 2) (all 2^23) for each of the divisors b in [1, 2) with
+// significands [b0, b0 + nb); x in pairs, both lanes.  Together with the
+// power-of-two scaling check below this covers the divider's stated range.
+__global__ void k_div_grid(uint32_t b0, uint32_t nb, unsigned long long* cnt, uint32_t* ex)
+{
+    const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+    const uint64_t total = (uint64_t)nb << 22;  // (b, x pair) items
+    for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
+        const uint32_t mb = b0 + (uint32_t)(i >> 22);
+        const uint32_t mx = (uint32_t)(i & ((1u << 22) - 1u)) << 1;
+        const float b = __uint_as_float(0x3F800000u | mb);
+        const float2 x = make_float2(__uint_as_float(0x3F800000u | mx), __uint_as_float(0x3F800000u | (mx + 1u)));
+        const float2 q = fo::div2_nr(x, make_float2(b, b), make_float2(-b, -b));
+        const bool bad0 = __float_as_uint(q.x) != __float_as_uint(__fdiv_rn(x.x, b));
+        const bool bad1 = __float_as_uint(q.y) != __float_as_uint(__fdiv_rn(x.y, b));
+        if (bad0 || bad1) {
+            const unsigned long long k = atomicAdd(&cnt[0], 1ull);
+            if (k < 2) {
+                ex[2 * k] = __float_as_uint(bad0 ? x.x : x.y);
+                ex[2 * k + 1] = __float_as_uint(b);
+            }
+        }
+    }
+}
+
+// cnt[0]: rcp_approx(b 2^e) != rcp_approx(b) 2^-e for a binary32 b in [1, 2)
+// and an exponent e in [-61, 61] (the approximate reciprocal scales exactly by
+// powers of two there); cnt[1]: the same for rsqrt_approx(b 2^(2e)) =
+// rsqrt_approx(b) 2^-e, e in [-30, 30]
+__global__ void k_rcp_scaling(unsigned long long* cnt, uint32_t* ex)
+{
+    const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+    for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (1ull << 23) * 123ull; i += stride) {
+        const uint32_t m = (uint32_t)(i % (1ull << 23));
+        const int e = (int)(i / (1ull << 23)) - 61;
+        const float b = __uint_as_float(0x3F800000u | m);
+        const float be = __uint_as_float((uint32_t)(127 + e) << 23 | m);
+        const float r = fo::rcp_approx(b), re = fo::rcp_approx(be);
+        if (__float_as_uint(re) != __float_as_uint(__fmul_rn(r, __uint_as_float((uint32_t)(127 - e) << 23))))
+            note(cnt, ex, 0, __float_as_uint(be));
+        if (e >= -30 && e <= 30) {
+            const float b2 = __uint_as_float((uint32_t)(127 + 2 * e) << 23 | m);
+            const float s = fo::rsqrt_approx(b), s2 = fo::rsqrt_approx(b2);
+            if (__float_as_uint(s2) != __float_as_uint(__fmul_rn(s, __uint_as_float((uint32_t)(127 - e) << 23))))
+                note(cnt, ex, 1, __float_as_uint(b2));
+        }
+    }
+}
+
 int launch_done(unsigned long long* hcnt, uint32_t* hex, unsigned long long* dcnt, uint32_t* dex)
 {
     if (cudaGetLastError() != cudaSuccess) return 2;
@@ -193,7 +243,9 @@ int launch_done(unsigned long long* hcnt, uint32_t* hex, unsigned long long* dcn
 }  // namespace
 
 // which: 0 ftz forms, 1 square root, 2 division (n pairs, seed), 3 rcp bound
-// and scale reciprocals, 4 / 5 fast bf16 / fp16 ECC8 codec.  cnt: 4 counters, ex: 16 example words (host memory).
+// and scale reciprocals, 4 / 5 fast bf16 / fp16 ECC8 codec, 6 division over
+// the significand grid (n divisor significands from seed), 7 power-of-two
+// scaling of the approximate reciprocal and reciprocal square root.  cnt: 4 counters, ex: 16 example words (host memory).
 extern "C" __attribute__((visibility("default"))) int fo_arith_check(int which, uint64_t n, uint64_t seed,
                                                                      unsigned long long* cnt, uint32_t* ex)
 {
@@ -214,6 +266,17 @@ extern "C" __attribute__((visibility("default"))) int fo_arith_check(int which, 
     case 3: k_rcp_scales<<<grid, block>>>(dcnt, dex); break;
     case 4: k_codec<0><<<grid, block>>>(dcnt, dex); break;
     case 5: k_codec<1><<<grid, block>>>(dcnt, dex); break;
+    case 6:
+        // divisor significands [seed, seed + n) (n <= 2^23 - seed; a slice per
+        // call keeps each launch short)
+        if (seed >= (1ull << 23) || n == 0 || n > (1ull << 23) - seed) {
+            cudaFree(dcnt);
+            cudaFree(dex);
+            return 5;
+        }
+        k_div_grid<<<grid, block>>>((uint32_t)seed, (uint32_t)n, dcnt, dex);
+        break;
+    case 7: k_rcp_scaling<<<grid, block>>>(dcnt, dex); break;
     default: break;
     }
     const int rc = launch_done(cnt, ex, dcnt, dex);

@@ -12,6 +12,12 @@ the IEEE operations of the exact path):
   compander's tie margin is derived from), the group-scale reciprocals
   equal 1/S and 255/S by div.rn for every finite fp16 scale S >= 0, and the
   computed variance-code values equal q/255 by div.rn for every code;
+* (opt-in, FO_EXHAUSTIVE=1, about a minute) the Newton-Raphson quotient equals
+  div.rn on every pair of significands (x, b in [1, 2): 2^46 pairs), and the
+  approximate reciprocal (reciprocal square root) scales exactly by powers of
+  two over the exponents the divider's range reaches: every correctly
+  rounded step of the divider then commutes with the scaling while its
+  intermediates stay normal, which extends the grid to the stated range;
 * the fast ECC8 codec of 16-bit masters (bit arithmetic; for fp16 an exact
   fma at and below the smallest normal) equals the exact codec: decode of
   every finite 16-bit pattern with every code, encode of every binary32 below
@@ -63,3 +69,23 @@ def test_fast_ecc8_codec_exhaustive(which, name):
     cnt, ex = arith_check.run(which)
     assert cnt[0] == 0, f"{name} decode differs on {cnt[0]} (x', code) pairs, e.g. {[hex(v) for v in ex[:4]]}"
     assert cnt[1] == 0, f"{name} encode differs on {cnt[1]} inputs, e.g. {[hex(v) for v in ex[4:8]]}"
+
+
+def test_approximations_scale_by_powers_of_two():
+    cnt, ex = arith_check.run(7)
+    assert cnt[0] == 0, f"rcp.approx does not scale on {cnt[0]} inputs, e.g. {[hex(v) for v in ex[:4]]}"
+    assert cnt[1] == 0, f"rsqrt.approx does not scale on {cnt[1]} inputs, e.g. {[hex(v) for v in ex[4:8]]}"
+
+
+@pytest.mark.exhaustive
+def test_newton_raphson_quotient_every_significand_pair():
+    """2^46 pairs in slices of 2^16 divisors (2^39 pairs, well under a second
+    per launch)."""
+    total, first = 0, None
+    step = 1 << 16
+    for b0 in range(0, 1 << 23, step):
+        cnt, ex = arith_check.run(6, n=step, seed=b0)
+        total += cnt[0]
+        if cnt[0] and first is None:
+            first = [hex(v) for v in ex[:4]]
+    assert total == 0, f"quotient differs on {total} significand pairs, e.g. (x, b) = {first}"
