@@ -98,44 +98,26 @@ struct StepLaunch {
     int threads;    // threads per block
     int smem;       // dynamic shared memory per block (stage buffers)
     int64_t chunk;  // elements per chunk
+    int ecc_bits;
 };
 
-template <int WDT, int GDT, int NB, int KIND, bool WIDE>
+template <int WDT, int GDT, int NB, int KIND>
 StepLaunch step_launch()
 {
-    using G = fo::Geometry<NB, KIND, WIDE>;
-    return {fo::step_kernel<WDT, GDT, NB, KIND, WIDE>, G::kBlockThreads, fo::step_smem_bytes<NB, KIND, WIDE>(),
-            G::kChunk};
-}
-
-// the geometry for a call over `total` elements: wide chunks for AdamW with
-// 8-bit ECC codes once the call is large enough
-template <int WDT, int GDT, int NB, int KIND>
-StepLaunch sized_launch(int64_t total)
-{
-    if constexpr (NB == 8 && fo::uses_v(KIND)) {
-        if (total >= fo::kWideMinElems) return step_launch<WDT, GDT, NB, KIND, true>();
-    }
-    return step_launch<WDT, GDT, NB, KIND, false>();
-}
-
-int64_t total_numel(const fo_tensor* t, int n)
-{
-    int64_t s = 0;
-    for (int i = 0; i < n; i++) s += t[i].numel;
-    return s;
+    using G = fo::Geometry<NB, KIND>;
+    return {fo::step_kernel<WDT, GDT, NB, KIND>, G::kBlockThreads, G::kSmemBytes, G::kChunk, NB};
 }
 
 // the step kernel of a format (k = nullptr if the format is not provided)
 template <int KIND>
-StepLaunch pick_step(const fo_format& f, int64_t total)
+StepLaunch pick_step(const fo_format& f)
 {
 #define FO_PICK(W, G, N)                                                                  \
-    if (f.w_dtype == W && f.grad_dtype == G && f.ecc_bits == N) return sized_launch<W, G, N, KIND>(total);
+    if (f.w_dtype == W && f.grad_dtype == G && f.ecc_bits == N) return step_launch<W, G, N, KIND>();
     FO_PICK(0, 0, 8) FO_PICK(0, 1, 8) FO_PICK(1, 0, 8) FO_PICK(1, 1, 8)
     FO_PICK(0, 0, 16) FO_PICK(0, 1, 16) FO_PICK(1, 0, 16) FO_PICK(1, 1, 16)
 #undef FO_PICK
-    return {nullptr, 0, 0, 0};
+    return {nullptr, 0, 0, 0, 0};
 }
 
 struct LaunchCache {
@@ -210,10 +192,17 @@ fo_status launch_step(const StepLaunch& L, const fo::Scalars& sc, const fo_tenso
             d.vq = x.v_q;
             d.vs = x.v_scale;
             d.numel = x.numel;
+            // staged chunks: every array 16-byte aligned (bulk copies, 128-bit
+            // stores) and the arrays written with 256-bit stores (weights, 16-bit
+            // ECC codes, with 16 elements per lane) 32-byte aligned; other
+            // tensors take the scalar path
             const uintptr_t a = (uintptr_t)x.w | (uintptr_t)x.grad | (uintptr_t)x.ecc | (uintptr_t)x.m_q |
                                 (uintptr_t)x.m_scale | (uintptr_t)x.v_q | (uintptr_t)x.v_scale;
+            const uintptr_t a32 = fo::kStagedElems == 16 ? ((uintptr_t)x.w | (L.ecc_bits == 16 ? (uintptr_t)x.ecc : 0)) : 0;
             d.n_chunks = (int32_t)((x.numel + chunk - 1) / chunk);
-            d.n_staged = (a & 15u) == 0 ? (int32_t)(x.numel / chunk) : 0;
+            d.staged = ((a & 15u) == 0 && (a32 & 31u) == 0) ? 1 : 0;
+            const int64_t last = x.numel - (int64_t)(d.n_chunks - 1) * chunk;  // elements of the last chunk
+            d.last_slices = (int16_t)(last / fo::kSlice);
             chunks += d.n_chunks;
             P.chunk_start[++m] = chunks;
         }
@@ -303,7 +292,8 @@ fo_status fo_adamw_step(const fo_tensor* t, int n_tensors, fo_format f, const fo
     sc.s[6] = (float)h->eps;
     sc.s[7] = (float)(1.0 - h->lr * h->weight_decay);
     adamw_fast_bounds(sc);
-    const StepLaunch L = pick_step<fo::kAdamW>(f, total_numel(t, n_tensors));
+    fo::fill_pairs(sc, true);
+    const StepLaunch L = pick_step<fo::kAdamW>(f);
     if (!L.k) return fail(FO_ERR_UNSUPPORTED, "format not provided");
     return launch_step(L, sc, t, n_tensors, (cudaStream_t)stream);
 }
@@ -332,7 +322,8 @@ fo_status fo_sgdm_step(const fo_tensor* t, int n_tensors, fo_format f, const fo_
     sc.s[5] = h->step == 1 ? 1.0f : 0.0f;
     sc.s[6] = 0.0f;
     sc.s[7] = 0.0f;
-    const StepLaunch L = pick_step<fo::kSGDM>(f, total_numel(t, n_tensors));
+    fo::fill_pairs(sc, false);
+    const StepLaunch L = pick_step<fo::kSGDM>(f);
     if (!L.k) return fail(FO_ERR_UNSUPPORTED, "format not provided");
     return launch_step(L, sc, t, n_tensors, (cudaStream_t)stream);
 }
@@ -347,12 +338,11 @@ fo_status fo_stream_copy(const fo_tensor* t, int n_tensors, fo_format f, int ada
     if (n_tensors == 0) return FO_OK;
     fo::Scalars sc = {};
     // the copy moves bytes only: the 16-bit formats do not matter, the ECC width does
-    const int64_t total = total_numel(t, n_tensors);
     StepLaunch L;
     if (adamw_mix)
-        L = f.ecc_bits == 8 ? sized_launch<0, 0, 8, fo::kCopyAdamW>(total) : sized_launch<0, 0, 16, fo::kCopyAdamW>(total);
+        L = f.ecc_bits == 8 ? step_launch<0, 0, 8, fo::kCopyAdamW>() : step_launch<0, 0, 16, fo::kCopyAdamW>();
     else
-        L = f.ecc_bits == 8 ? sized_launch<0, 0, 8, fo::kCopySGDM>(total) : sized_launch<0, 0, 16, fo::kCopySGDM>(total);
+        L = f.ecc_bits == 8 ? step_launch<0, 0, 8, fo::kCopySGDM>() : step_launch<0, 0, 16, fo::kCopySGDM>();
     return launch_step(L, sc, t, n_tensors, (cudaStream_t)stream);
 }
 
@@ -411,6 +401,22 @@ fo_status fo_decode_master(const void* w, const void* ecc, float* x32, int64_t n
     return e == cudaSuccess ? FO_OK : cuda_fail(e, "decode kernel launch");
 }
 
+fo_status fo_check_errors(void* stream)
+{
+    g_last_error.clear();
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    unsigned int n = 0;
+    e = cudaMemcpyFromSymbol(&n, fo::g_wait_timeouts, sizeof n);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyFromSymbol");
+    if (n == 0) return FO_OK;
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(fo::g_wait_timeouts, &zero, sizeof zero);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyToSymbol");
+    return fail(FO_ERR_TIMEOUT, std::to_string(n) + " warp(s) gave up waiting for a staged copy; their chunks were "
+                                                    "not stepped");
+}
+
 const char* fo_status_string(fo_status s)
 {
     switch (s) {
@@ -420,12 +426,13 @@ const char* fo_status_string(fo_status s)
     case FO_ERR_ALIGNMENT: return "FO_ERR_ALIGNMENT";
     case FO_ERR_TOO_MANY_TENSORS: return "FO_ERR_TOO_MANY_TENSORS";
     case FO_ERR_CUDA: return "FO_ERR_CUDA";
+    case FO_ERR_TIMEOUT: return "FO_ERR_TIMEOUT";
     }
     return "unknown fo_status";
 }
 
 const char* fo_last_error(void) { return g_last_error.c_str(); }
 
-int fo_version(void) { return 100; }
+int fo_version(void) { return 200; }
 
 }  // extern "C"

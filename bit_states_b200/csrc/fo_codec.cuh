@@ -16,6 +16,7 @@
 // round-half-even to integer) and integer bit arithmetic are used.
 #pragma once
 
+#include <cstddef>
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>

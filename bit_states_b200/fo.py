@@ -49,7 +49,7 @@ class fo_format(ctypes.Structure):
 
 
 EXPORTS = ("fo_adamw_step", "fo_sgdm_step", "fo_stream_copy", "fo_encode_master", "fo_decode_master",
-           "fo_status_string", "fo_last_error", "fo_version")
+           "fo_check_errors", "fo_status_string", "fo_last_error", "fo_version")
 
 _lib = None
 
@@ -70,7 +70,9 @@ def load(path: str = LIB_PATH):
     lib.fo_stream_copy.argtypes = [ctypes.POINTER(fo_tensor), I, fo_format, I, P]
     lib.fo_encode_master.argtypes = [P, P, P, I64, fo_format, P]
     lib.fo_decode_master.argtypes = [P, P, P, I64, fo_format, P]
-    for n in ("fo_adamw_step", "fo_sgdm_step", "fo_stream_copy", "fo_encode_master", "fo_decode_master"):
+    lib.fo_check_errors.argtypes = [P]
+    for n in ("fo_adamw_step", "fo_sgdm_step", "fo_stream_copy", "fo_encode_master", "fo_decode_master",
+              "fo_check_errors"):
         getattr(lib, n).restype = I
     lib.fo_status_string.argtypes = [I]
     lib.fo_status_string.restype = ctypes.c_char_p
@@ -157,6 +159,12 @@ def fo_encode_master(x32, w, ecc, n: int, fmt: fo_format, stream=None):
 def fo_decode_master(w, ecc, x32, n: int, fmt: fo_format, stream=None):
     _check(load().fo_decode_master(_ptr(w), _ptr(ecc), _ptr(x32), int(n), fmt, _stream_handle(stream)),
            "fo_decode_master")
+
+
+def fo_check_errors(stream=None):
+    """Wait for ``stream`` and raise if a step kernel gave up a bounded wait
+    for a staged copy since the last check (its chunks were not stepped)."""
+    _check(load().fo_check_errors(_stream_handle(stream)), "fo_check_errors")
 
 
 def fo_version() -> int:

@@ -61,10 +61,14 @@
  *   - numel == 0 tensors are skipped; n_tensors == 0 is a no-op.
  *   - Results do not depend on the number of tensors per call, their order,
  *     or on whether they are stepped in one call or one call per tensor.
- *   - Launch geometry (performance only, results identical): AdamW calls with
- *     8-bit ECC codes over at least 3 * 2^25 elements in total use chunks of 768
- *     elements in 10-warp blocks, every other call chunks of 512 elements in
- *     8-warp blocks; a tensor's last partial chunk takes the scalar path.
+ *   - Launch geometry (performance only, results identical): chunks of 1024
+ *     elements (512 where the stage buffers would not fit), staged in shared
+ *     memory by bulk copies, one warp per chunk; the elements of a tensor's
+ *     last chunk beyond its whole 512-element slices, and tensors whose
+ *     arrays are not 16-byte aligned (or whose weights / 16-bit ECC codes are
+ *     not 32-byte aligned), take a scalar path.
+ *   - Waits inside the kernels are bounded in time; fo_check_errors reports
+ *     a wait that gave up.
  */
 #ifndef FO_H
 #define FO_H
@@ -87,7 +91,8 @@ typedef enum {
     FO_ERR_UNSUPPORTED = 2,      /* dtype / ecc_bits combination not provided */
     FO_ERR_ALIGNMENT = 3,        /* a 16-bit array not 2-byte aligned */
     FO_ERR_TOO_MANY_TENSORS = 4, /* n_tensors above FO_MAX_TENSORS_PER_CALL */
-    FO_ERR_CUDA = 5              /* a CUDA runtime call or launch failed */
+    FO_ERR_CUDA = 5,             /* a CUDA runtime call or launch failed */
+    FO_ERR_TIMEOUT = 6           /* a kernel gave up a bounded wait (fo_check_errors) */
 } fo_status;
 
 typedef enum { FO_DT_BF16 = 0, FO_DT_FP16 = 1 } fo_dtype;
@@ -207,6 +212,17 @@ FO_API fo_status fo_encode_master(const float* x32, void* w, void* ecc, int64_t 
  */
 FO_API fo_status fo_decode_master(const void* w, const void* ecc, float* x32, int64_t n, fo_format f,
                            void* stream);
+
+/*
+ * fo_check_errors - wait for the work on `stream` (a cudaStream_t), then
+ * report whether any step kernel on the current device gave up a bounded
+ * wait for one of its staged copies since the last check.  Such a kernel
+ * leaves the chunks of the warp that gave up unstepped (their bytes are
+ * unspecified); this never happens on a healthy device.  Returns FO_OK, or
+ * FO_ERR_TIMEOUT (and clears the device's count), or FO_ERR_CUDA.
+ * Passage: none (error reporting).
+ */
+FO_API fo_status fo_check_errors(void* stream);
 
 /* Static English name of a status code.  Passage: none (error reporting). */
 FO_API const char* fo_status_string(fo_status s);

@@ -45,6 +45,7 @@ def test_version_and_status_strings(lib):
     assert lib.fo_version() >= 100
     assert lib.fo_status_string(0) == b"FO_OK"
     assert lib.fo_status_string(5) == b"FO_ERR_CUDA"
+    assert lib.fo_status_string(6) == b"FO_ERR_TIMEOUT"
 
 
 def _hp(**kw):

@@ -89,3 +89,4 @@ def test_newton_raphson_quotient_every_significand_pair():
         if cnt[0] and first is None:
             first = [hex(v) for v in ex[:4]]
     assert total == 0, f"quotient differs on {total} significand pairs, e.g. (x, b) = {first}"
+

@@ -154,7 +154,8 @@ def test_flat_1m_ten_adamw_steps_every_byte():
 
 # ---- ragged sizes, misaligned views, all formats ------------------------------------
 
-RAGGED = [1, 2, 31, 32, 33, 255, 256, 257, 511, 512, 513, 767, 768, 769, 1000, 1536, 1537, 4095, 4096, 65537]
+RAGGED = [1, 2, 31, 32, 33, 255, 256, 257, 511, 512, 513, 767, 768, 769, 1000, 1023, 1024, 1025, 1536, 1537,
+          2047, 2048, 2049, 2560, 2561, 3071, 3072, 3073, 4095, 4096, 65537]
 
 
 def _ragged_workload(opt, wdt, gdt, nbits):
@@ -172,20 +173,20 @@ def test_ragged_multitensor_all_formats(opt, wdt, gdt, nbits):
     _run_full_compare(wl, 3)
 
 
-# calls of AdamW with 8-bit ECC codes over at least 3 * 2^25 elements take
-# the wide launch geometry (chunks of 768 elements in 10-warp blocks)
-WIDE_MIN = 3 << 25
+# a tensor large enough that every warp of the persistent grid walks many
+# chunks of it
+LARGE = 3 << 25
 
 
 @pytest.mark.parametrize("wdt,gdt", [("bf16", "bf16"), ("fp16", "fp16"), ("bf16", "fp16"), ("fp16", "bf16")])
-def test_ragged_wide_geometry(wdt, gdt):
-    """The ragged list plus one tensor of 3 * 2^25 + 45 elements: the call is
-    large enough for the wide geometry, so every tensor (ragged tails, chunk
-    edges at 767 / 768 / 769 and 1536 / 1537) goes through it; every byte of
-    every ragged tensor and sampled groups of the large one against the
-    oracle."""
+def test_ragged_with_large_tensor(wdt, gdt):
+    """The ragged list plus one tensor of 3 * 2^25 + 45 elements in the middle:
+    every warp walks many chunks, across tensor boundaries (ragged tails,
+    slice and chunk edges at 511 / 512 / 513, 1023 / 1024 / 1025 and
+    1535 / 1536 / 1537); every byte of every
+    ragged tensor and sampled groups of the large one against the oracle."""
     wl = _ragged_workload("adamw", wdt, gdt, 8)
-    wl.tensors.insert(7, TensorSpec("fill", (WIDE_MIN + 45,), "normal", 0.02))
+    wl.tensors.insert(7, TensorSpec("fill", (LARGE + 45,), "normal", 0.02))
     _run_full_compare(wl, 2, sample_above=1 << 20)
 
 
@@ -207,25 +208,32 @@ def test_sgdm_variants(nesterov, damp):
     _run_full_compare(wl, 3)
 
 
-@pytest.mark.parametrize("shift", [1, 2, 3, 8, 16])
-def test_misaligned_views_take_scalar_path(shift):
-    """Tensors whose arrays start off the 32-byte grid (views into a larger
-    buffer) give the same bytes; canaries around every output stay intact."""
+@pytest.mark.parametrize("nbits", [8, 16])
+@pytest.mark.parametrize("s16,s8", [(1, 1), (2, 2), (3, 3), (8, 8), (16, 16), (8, 16), (24, 32), (16, 16 + 8)])
+def test_misaligned_views_take_scalar_path(s16, s8, nbits):
+    """Tensors whose arrays start off the 16-byte grid, or whose weights (and
+    16-bit ECC codes) start off the 32-byte grid that their 256-bit stores
+    need, take the scalar path; arrays on both grids take the staged path.
+    Views into larger buffers: the 16-bit arrays are shifted by s16 elements,
+    the 8-bit ones by s8.  Same bytes as the oracle either way, and canaries
+    around every output stay intact."""
     n = 3000
-    wl = _ragged_workload("adamw", "bf16", "bf16", 8)
+    wl = _ragged_workload("adamw", "bf16", "bf16", nbits)
     wl.tensors = [TensorSpec("a", (n,), "normal", 0.02)]
     idx = np.arange(n)
     x = wl.master_values(0, idx)
-    ow, oe = oracle.encode_master(x, 0, 8)
+    ow, oe = oracle.encode_master(x, 0, nbits)
     pad = 64
     mk = lambda dt, cnt: torch.full((cnt + 2 * pad,), 0x5A, dtype=dt, device=DEV)
-    w = mk(torch.int16, n); e = mk(torch.int8, n); mq = mk(torch.int8, n); vq = mk(torch.uint8, n)
+    edt = torch.int8 if nbits == 8 else torch.int16
+    w = mk(torch.int16, n); e = mk(edt, n); mq = mk(torch.int8, n); vq = mk(torch.uint8, n)
     ng = (n + 31) // 32
     ms = mk(torch.int16, ng); vs = mk(torch.int16, ng); g = mk(torch.int16, n)
-    s = shift
-    wv, ev, mqv, vqv, gv = w[pad + s:pad + s + n], e[pad + s:pad + s + n], mq[pad + s:pad + s + n], \
-        vq[pad + s:pad + s + n], g[pad + s:pad + s + n]
-    msv, vsv = ms[pad + 1:pad + 1 + ng], vs[pad + 1:pad + 1 + ng]
+    se = s8 if nbits == 8 else s16
+    shifts = dict(w=s16, e=se, mq=s8, vq=s8, g=s16, ms=8, vs=8)
+    views = {k: full[pad + shifts[k]:pad + shifts[k] + (ng if k in ("ms", "vs") else n)]
+             for k, full in dict(w=w, e=e, mq=mq, vq=vq, g=g, ms=ms, vs=vs).items()}
+    wv, ev, mqv, vqv, gv, msv, vsv = (views[k] for k in ("w", "e", "mq", "vq", "g", "ms", "vs"))
     wv.copy_(torch.from_numpy(ow.view(np.int16))); ev.copy_(torch.from_numpy(oe))
     mqv.zero_(); vqv.zero_(); msv.zero_(); vsv.zero_()
     st = oracle.State.zeros_like_master(ow, oe)
@@ -235,8 +243,8 @@ def test_misaligned_views_take_scalar_path(shift):
         gb = wl.grad_bits(0, t, idx)
         gv.copy_(torch.from_numpy(gb.view(np.int16)))
         d = fo.descriptors([state], [gv])
-        fo.fo_adamw_step(d, 1, fo.make_format(), U.hparams_adamw(wl, t))
-        oracle.adamw_step(st, gb, **wl.hparams, step=t)
+        fo.fo_adamw_step(d, 1, fo.make_format("bf16", "bf16", nbits), U.hparams_adamw(wl, t))
+        oracle.adamw_step(st, gb, **wl.hparams, step=t, ecc_bits=nbits)
     torch.cuda.synchronize()
     assert np.array_equal(U.to_np_bytes(wv), st.w)
     assert np.array_equal(ev.cpu().numpy(), st.ecc)
@@ -245,10 +253,11 @@ def test_misaligned_views_take_scalar_path(shift):
     assert np.array_equal(U.to_np_bytes(msv), st.ms)
     assert np.array_equal(U.to_np_bytes(vsv), st.vs)
     for k, full in dict(w=w, e=e, mq=mq, vq=vq, ms=ms, vs=vs).items():
-        lo = pad + (1 if k in ("ms", "vs") else s)
+        lo = pad + shifts[k]
         cnt = ng if k in ("ms", "vs") else n
         assert torch.equal(full[:lo], before[k][:lo]), k
         assert torch.equal(full[lo + cnt:], before[k][lo + cnt:]), k
+    fo.fo_check_errors()
 
 
 def test_empty_and_tiny_tensors_in_one_call():
@@ -270,11 +279,11 @@ def test_empty_and_tiny_tensors_in_one_call():
         assert all(v == 0 for v in U.mismatches(exp, U.gather_device(P, ti, exp)).values())
 
 
-@pytest.mark.parametrize("fill", [0, WIDE_MIN])
+@pytest.mark.parametrize("fill", [0, LARGE])
 def test_many_tensors_split_across_launches(fill):
     """1000 tensors in one call: more than one launch's parameter block holds
     (384 descriptors), so the call is split into several launches (with a
-    3 * 2^25-element tensor in the middle, all of them in the wide geometry).
+    3 * 2^25-element tensor in the middle).
     Every byte of every tensor (sampled groups of the large one) against the
     oracle."""
     rng = np.random.default_rng(17)
