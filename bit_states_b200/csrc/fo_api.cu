@@ -99,13 +99,14 @@ struct StepLaunch {
     int smem;       // dynamic shared memory per block (stage buffers)
     int64_t chunk;  // elements per chunk
     int ecc_bits;
+    int lane;       // elements per lane in a staged slice
 };
 
 template <int WDT, int GDT, int NB, int KIND>
 StepLaunch step_launch()
 {
     using G = fo::Geometry<NB, KIND>;
-    return {fo::step_kernel<WDT, GDT, NB, KIND>, G::kBlockThreads, G::kSmemBytes, G::kChunk, NB};
+    return {fo::step_kernel<WDT, GDT, NB, KIND>, G::kBlockThreads, G::kSmemBytes, G::kChunk, NB, G::kLane};
 }
 
 // the step kernel of a format (k = nullptr if the format is not provided)
@@ -117,7 +118,7 @@ StepLaunch pick_step(const fo_format& f)
     FO_PICK(0, 0, 8) FO_PICK(0, 1, 8) FO_PICK(1, 0, 8) FO_PICK(1, 1, 8)
     FO_PICK(0, 0, 16) FO_PICK(0, 1, 16) FO_PICK(1, 0, 16) FO_PICK(1, 1, 16)
 #undef FO_PICK
-    return {nullptr, 0, 0, 0, 0};
+    return {nullptr, 0, 0, 0, 0, 0};
 }
 
 struct LaunchCache {
@@ -198,11 +199,11 @@ fo_status launch_step(const StepLaunch& L, const fo::Scalars& sc, const fo_tenso
             // tensors take the scalar path
             const uintptr_t a = (uintptr_t)x.w | (uintptr_t)x.grad | (uintptr_t)x.ecc | (uintptr_t)x.m_q |
                                 (uintptr_t)x.m_scale | (uintptr_t)x.v_q | (uintptr_t)x.v_scale;
-            const uintptr_t a32 = fo::kStagedElems == 16 ? ((uintptr_t)x.w | (L.ecc_bits == 16 ? (uintptr_t)x.ecc : 0)) : 0;
+            const uintptr_t a32 = L.lane == 16 ? ((uintptr_t)x.w | (L.ecc_bits == 16 ? (uintptr_t)x.ecc : 0)) : 0;
             d.n_chunks = (int32_t)((x.numel + chunk - 1) / chunk);
             d.staged = ((a & 15u) == 0 && (a32 & 31u) == 0) ? 1 : 0;
             const int64_t last = x.numel - (int64_t)(d.n_chunks - 1) * chunk;  // elements of the last chunk
-            d.last_slices = (int16_t)(last / fo::kSlice);
+            d.last_slices = (int16_t)(last / (32 * L.lane));
             chunks += d.n_chunks;
             P.chunk_start[++m] = chunks;
         }

@@ -180,11 +180,25 @@ def llama31_8b(order: str = "forward", ecc_bits: int = 8) -> Workload:
     return wl
 
 
+def llama31_layers(n_layers: int = 2) -> Workload:
+    """The first decoder layers of the Llama-3.1-8B list (same shapes, values
+    and hyper-parameters as in the full list): a case of a few GB, far above
+    the L2, for profiler captures of the full-size kernel."""
+    full = llama31_8b()
+    per_layer = 9
+    ts = full.tensors[1:1 + per_layer * n_layers]
+    return Workload(
+        name=f"llama3.1-8b-{n_layers}layers", tensors=ts, optimizer="adamw", hparams=dict(ADAMW_HP),
+        grad_dist="student_t3", grad_scale=1e-4, warm_steps=0,
+        description=f"decoder layers 0..{n_layers - 1} of the Llama-3.1-8B parameter list")
+
+
 CONFIGS = {
     "flat-1M": flat_1m,
     "gpt2-small-124M": gpt2_small,
     "resnet50-25.6M": resnet50,
     "llama3.1-8b": llama31_8b,
+    "llama3.1-8b-2layers": llama31_layers,
 }
 
 
