@@ -9,9 +9,12 @@ far above the 126 MB L2, so no flush is needed between steps.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
     python bench.py --impl reference ...     # the CPU oracle, timed on host cores
 
-Prints one JSON line (rank 0).  Multi-GPU: one process per GPU (torchrun),
-each rank steps its own parameter shard of the same shape (weak scaling, no
-data-path collective); time = max over ranks of the device-event time.
+Prints one JSON line (rank 0).  Multi-GPU: one process per GPU (torchrun);
+by default the list is sharded over the ranks as in data-parallel training
+(--mode dp: NCCL reduce-scatter of the gradients, the fused step on each
+rank's groups, all-gather of x'; strong scaling), or every rank steps its own
+copy (--mode replicas: weak scaling, no data-path collective); time = max
+over ranks of the device-event time.
 """
 from __future__ import annotations
 
@@ -46,6 +49,14 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-params", type=int, default=1 << 24)
     ap.add_argument("--launch-mode", default="multi", choices=["multi", "release"])
+    ap.add_argument("--mode", default=None, choices=["fused", "dp", "replicas"],
+                    help="fused: one GPU steps the whole list (default for one GPU); dp: the list is sharded "
+                         "over the ranks, one step = NCCL reduce-scatter of the 16-bit gradients, the fused "
+                         "step on each rank's groups, all-gather of x' (default for several GPUs); replicas: "
+                         "every rank steps its own copy of the list, no collective")
+    ap.add_argument("--bucket-groups", type=int, default=1 << 22,
+                    help="groups of 32 elements per data-parallel bucket (2^22: 128M parameters, 256 MB of "
+                         "16-bit gradients)")
     ap.add_argument("--flush-l2", action="store_true",
                     help="write a 512 MB buffer before every timed step and time each step's kernels alone "
                          "(for workloads that fit in the 126 MB L2)")
@@ -280,8 +291,12 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.mode is None:
+        args.mode = "dp" if world > 1 else "fused"
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.mode == "dp":
+        return run_dp(args, rank, world, local)
 
     import torch
 
@@ -507,6 +522,191 @@ def main():
     if dist:
         dist.barrier()
         dist.destroy_process_group()
+    return 0
+
+
+def _free_port() -> int:
+    import socket
+
+    so = socket.socket()
+    so.bind(("127.0.0.1", 0))
+    port = so.getsockname()[1]
+    so.close()
+    return port
+
+
+def run_dp(args, rank, world, local):
+    """Data-parallel step of one model over `world` GPUs (strong scaling: the
+    list is the same for every N).  The flat layout of the parameter list is
+    cut into buckets; rank r owns the r-th slice of every bucket (its ECC,
+    momentum and variance codes and scales) and holds the whole x'.  One step:
+    NCCL reduce-scatter of the 16-bit gradients, the fused step of the owned
+    slices, all-gather of x' in place, bucket by bucket on a communication
+    stream (bit_states_b200.dp).  Rank 0 holds the synthetic gradient and the
+    other ranks zeros, so the reduced gradient is rank 0's exactly, in any
+    summation order.  Also timed: the steps alone and the exchange alone."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    if not torch.cuda.is_available():
+        print(json.dumps({"metric": METRIC, "error": "no CUDA device"}), flush=True)
+        return 1
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    else:
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0, world_size=1,
+                                timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    from bit_states_b200 import build as fobuild
+    from bit_states_b200 import fo
+    from bit_states_b200.dp import DataParallelStep, FlatLayout, ShardedState
+    from workloads import device as wdev
+    from workloads import workload
+
+    fobuild.build()
+    wdev.build()
+    fo.load()
+    wl = workload(args.config)
+    adam = wl.optimizer == "adamw"
+    layout = FlatLayout([t.numel for t in wl.tensors], world, bucket_groups=args.bucket_groups)
+    st = ShardedState(layout, rank, dev, adam=adam, ecc_bits=wl.ecc_bits)
+    fmt = fo.make_format(wl.w_dtype, wl.grad_dtype, wl.ecc_bits)
+    # masters: the same synthetic values on every rank, encoded by the owner
+    # of each group and all-gathered
+    x32 = torch.zeros(layout.numel, dtype=torch.float32, device=dev)
+    for ti, t in enumerate(wl.tensors):
+        wdev.master_f32(wl, ti, layout.tensor_view(x32, ti))
+    st.encode_from(x32, fmt, w_dtype=wl.w_dtype)
+    del x32
+    grads = torch.zeros(layout.numel, dtype=torch.int16, device=dev)
+    if rank == 0:
+        for ti in range(len(wl.tensors)):
+            wdev.grad_16(wl, ti, 1, layout.tensor_view(grads, ti))
+    h = wl.hparams
+    dp = DataParallelStep(st, fmt=fmt, hparams=h, reduce_op="sum", grad_dtype=wl.grad_dtype,
+                          w_dtype=wl.w_dtype, optimizer=wl.optimizer)
+    torch.cuda.synchronize()
+    dist.barrier()
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, k):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        dist.barrier()
+        e0.record(stream)
+        for _ in range(k):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dist.barrier()
+        tt = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        return float(tt[0]) / k
+
+    t = [0]
+
+    def one_step():
+        t[0] += 1
+        dp.step(grads, t[0])
+
+    def step_only():
+        t[0] += 1
+        dp.step_only(t[0], stream)
+
+    for _ in range(args.warmup):
+        one_step()
+    gpu_id = "0"
+    try:
+        props = torch.cuda.get_device_properties(local)
+        gpu_id = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+    except Exception:
+        pass
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    K = args.steps
+    total_ms = timed(one_step, K)
+    clocks = sampler.stop()
+    fo.fo_check_errors()
+    step_ms = timed(step_only, max(3, K // 2))
+    comm_ms = timed(lambda: dp.exchange(grads), max(3, K // 2))
+    fo.fo_check_errors()
+
+    n_params = wl.numel
+    value = n_params / (total_ms / 1e3) / 1e9
+    owned = st.m_q.numel()
+    per_param = algorithmic_bytes(wl) / n_params
+    step_bytes = per_param * owned
+    peak, peak_kind = measured_peaks()
+    achieved = step_bytes / (step_ms / 1e3) / 1e9
+    overlap = (step_ms + comm_ms - total_ms) / min(step_ms, comm_ms) if min(step_ms, comm_ms) > 0 else None
+
+    # end to end through the public API: every step copies this rank's
+    # gradient from pinned host memory (in pieces) and reads x' back
+    PIECE = 1 << 24
+    host_g = torch.empty(PIECE, dtype=torch.int16, pin_memory=True)
+    host_g.copy_(grads[:PIECE].cpu() if layout.numel >= PIECE else torch.zeros(PIECE, dtype=torch.int16))
+    host_w = torch.empty(PIECE, dtype=torch.int16, pin_memory=True)
+
+    def e2e_step():
+        for a in range(0, layout.numel, PIECE):
+            b = min(layout.numel, a + PIECE)
+            grads[a:b].copy_(host_g[:b - a], non_blocking=True)
+        one_step()
+        for a in range(0, layout.numel, PIECE):
+            b = min(layout.numel, a + PIECE)
+            host_w[:b - a].copy_(st.w[a:b], non_blocking=True)
+
+    e2e_steps = max(1, min(args.e2e_steps, 3))
+    e2e = None
+    if not args.no_e2e:
+        e2e_ms = timed(e2e_step, e2e_steps)
+        e2e = {"value": round(n_params / (e2e_ms / 1e3) / 1e9, 3), "unit": "Gparams/s",
+               "h2d_bytes_per_step": 2 * layout.numel, "d2h_bytes_per_step": 2 * layout.numel,
+               "ms_per_step": round(e2e_ms, 3), "steps": e2e_steps,
+               "how": f"per step and rank: the rank's 16-bit gradient from a pinned host buffer to the device in "
+                      f"pieces of {PIECE} elements, the data-parallel step, x' back to pinned host memory"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = os.cpu_count() or 1
+        v, dt, n, k = time_oracle(wl, args.cpu_sample_params, 1, 1, threads, min_seconds=10.0)
+        cpu = {"value": round(v, 6), "unit": "Gparams/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n} params (whole 32-groups drawn from all {len(wl.tensors)} tensors), "
+                         f"{k} {wl.optimizer} steps after one warm step, {threads} host threads, {dt:.2f} s timed"}
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": "Gparams/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": round(total_ms, 4), "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"{wl.name}: {len(wl.tensors)} tensors, {n_params} params in total, "
+                                   f"{wl.optimizer} {wl.w_dtype}+ecc{wl.ecc_bits}, int8/uint8 companded states",
+                       "launch": f"{len(layout.buckets)} buckets of <= {args.bucket_groups} groups; per bucket a "
+                                 "fused step on this rank's slice",
+                       "l2": "inputs larger than L2 (%.2f GB per step per GPU vs 126 MB)" % (step_bytes / 1e9),
+                       "parallelism": f"data parallel x{world}: NCCL reduce-scatter of 16-bit gradients, fused step "
+                                      f"on owned groups, in-place all-gather of x'"},
+            "exchange": {"total_ms": round(total_ms, 3), "steps_only_ms": round(step_ms, 3),
+                         "exchange_only_ms": round(comm_ms, 3),
+                         "overlap": None if overlap is None else round(overlap, 3),
+                         "bytes_per_rank": {"reduce_scatter_in": 2 * layout.numel * (world - 1) // world,
+                                            "all_gather_in": 2 * layout.numel * (world - 1) // world}},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": None, "peak_kind": peak_kind,
+                         "algorithmic_bytes_per_launch": int(step_bytes / max(1, len(layout.buckets))),
+                         "kernel": "fo::step_kernel (the owned slices' steps, timed without the exchange)"},
+            "clocks": clocks,
+            "gpu_launches": K * len(layout.buckets),
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    dist.barrier()
+    dist.destroy_process_group()
     return 0
 
 

@@ -91,10 +91,13 @@ fo_status check_tensors(const fo_tensor* t, int n, const fo_format& f, bool adam
 // ---- launch of one step over a tensor list -----------------------------------
 
 using StepKernel = void (*)(const fo::StepParams);
+using SmallStepKernel = void (*)(const fo::StepParamsT<fo::kSmallTensors>);
 
-// one step kernel with its launch geometry (fo::Geometry)
+// one step kernel (two parameter-table sizes) with its launch geometry
+// (fo::Geometry)
 struct StepLaunch {
     StepKernel k;
+    SmallStepKernel ks;
     int threads;    // threads per block
     int smem;       // dynamic shared memory per block (stage buffers)
     int64_t chunk;  // elements per chunk
@@ -106,7 +109,9 @@ template <int WDT, int GDT, int NB, int KIND>
 StepLaunch step_launch()
 {
     using G = fo::Geometry<NB, KIND>;
-    return {fo::step_kernel<WDT, GDT, NB, KIND>, G::kBlockThreads, G::kSmemBytes, G::kChunk, NB, G::kLane};
+    return {fo::step_kernel<WDT, GDT, NB, KIND, fo::kMaxTensorsPerLaunch>,
+            fo::step_kernel<WDT, GDT, NB, KIND, fo::kSmallTensors>,
+            G::kBlockThreads, G::kSmemBytes, G::kChunk, NB, G::kLane};
 }
 
 // the step kernel of a format (k = nullptr if the format is not provided)
@@ -118,7 +123,7 @@ StepLaunch pick_step(const fo_format& f)
     FO_PICK(0, 0, 8) FO_PICK(0, 1, 8) FO_PICK(1, 0, 8) FO_PICK(1, 1, 8)
     FO_PICK(0, 0, 16) FO_PICK(0, 1, 16) FO_PICK(1, 0, 16) FO_PICK(1, 1, 16)
 #undef FO_PICK
-    return {nullptr, 0, 0, 0, 0, 0};
+    return {nullptr, nullptr, 0, 0, 0, 0, 0};
 }
 
 struct LaunchCache {
@@ -131,7 +136,8 @@ struct LaunchCache {
 
 // once per (device, kernel): allow the dynamic shared memory of the stage
 // buffers and find how many blocks fit on one SM
-fo_status prepare_kernel(StepKernel k, int threads, int smem, int* blocks_per_sm)
+template <class KERNEL>
+fo_status prepare_kernel(KERNEL k, int threads, int smem, int* blocks_per_sm)
 {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -158,66 +164,94 @@ fo_status prepare_kernel(StepKernel k, int threads, int smem, int* blocks_per_sm
     return FO_OK;
 }
 
-fo_status launch_step(const StepLaunch& L, const fo::Scalars& sc, const fo_tensor* t, int n, cudaStream_t stream)
+// Pack up to MAXT tensors from t[i..] (skipping empty ones) into P and
+// launch; returns the index of the first tensor not packed.
+template <int MAXT, class KERNEL>
+fo_status launch_table(KERNEL kernel, const StepLaunch& L, const fo::Scalars& sc, const fo_tensor* t, int n,
+                       int& i, int64_t cap, cudaStream_t stream)
 {
     const int64_t chunk = L.chunk;
     const int warps = L.threads / 32;
-    bool any = false;
-    for (int j = 0; j < n && !any; j++) any = t[j].numel > 0;
-    if (!any) return FO_OK;
+    // kernel parameters are copied at launch, so one block of host memory
+    // per thread serves every launch
+    thread_local fo::StepParamsT<MAXT> P;
+    std::memset(&P, 0, offsetof(fo::StepParamsT<MAXT>, t));
+    P.sc = sc;
+    int m = 0;
+    int64_t chunks = 0;
+    P.chunk_start[0] = 0;
+    for (; i < n && m < MAXT; i++) {
+        const fo_tensor& x = t[i];
+        if (x.numel == 0) continue;
+        fo::TensorDesc& d = P.t[m];
+        d.w = x.w;
+        d.ecc = x.ecc;
+        d.grad = x.grad;
+        d.mq = x.m_q;
+        d.ms = x.m_scale;
+        d.vq = x.v_q;
+        d.vs = x.v_scale;
+        d.numel = x.numel;
+        // staged chunks: every array 16-byte aligned (bulk copies, 128-bit
+        // stores) and the arrays written with 256-bit stores (weights, 16-bit
+        // ECC codes, with 16 elements per lane) 32-byte aligned; other
+        // tensors take the scalar path
+        const uintptr_t a = (uintptr_t)x.w | (uintptr_t)x.grad | (uintptr_t)x.ecc | (uintptr_t)x.m_q |
+                            (uintptr_t)x.m_scale | (uintptr_t)x.v_q | (uintptr_t)x.v_scale;
+        const uintptr_t a32 = L.lane == 16 ? ((uintptr_t)x.w | (L.ecc_bits == 16 ? (uintptr_t)x.ecc : 0)) : 0;
+        d.n_chunks = (int32_t)((x.numel + chunk - 1) / chunk);
+        d.staged = ((a & 15u) == 0 && (a32 & 31u) == 0) ? 1 : 0;
+        const int64_t last = x.numel - (int64_t)(d.n_chunks - 1) * chunk;  // elements of the last chunk
+        d.last_slices = (int16_t)(last / (32 * L.lane));
+        chunks += d.n_chunks;
+        P.chunk_start[++m] = chunks;
+    }
+    if (m == 0) return FO_OK;
+    P.n_tensors = m;
+    P.total_chunks = chunks;
+    // a sentinel past the last tensor keeps the device-side walk bounded
+    for (int j = m + 1; j <= MAXT; j++) P.chunk_start[j] = INT64_MAX;
+    int64_t grid = (chunks + warps - 1) / warps;
+    if (grid > cap) grid = cap;
+    // programmatic stream serialization: the kernel may be scheduled while
+    // the previous kernel on the stream finishes; it waits for it
+    // (griddepcontrol.wait) before touching global memory
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)L.threads);
+    cfg.dynamicSmemBytes = (size_t)L.smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, P);
+    if (e != cudaSuccess) return cuda_fail(e, "step kernel launch");
+    return FO_OK;
+}
+
+fo_status launch_step(const StepLaunch& L, const fo::Scalars& sc, const fo_tensor* t, int n, cudaStream_t stream)
+{
+    int live = 0;
+    for (int j = 0; j < n; j++) live += t[j].numel > 0;
+    if (live == 0) return FO_OK;
     int sms = 0;
     fo_status st = device_sms(&sms);
     if (st != FO_OK) return st;
     int bps = 1;
+    if (live <= fo::kSmallTensors) {
+        st = prepare_kernel(L.ks, L.threads, L.smem, &bps);
+        if (st != FO_OK) return st;
+        int i = 0;
+        return launch_table<fo::kSmallTensors>(L.ks, L, sc, t, n, i, (int64_t)sms * bps, stream);
+    }
     st = prepare_kernel(L.k, L.threads, L.smem, &bps);
     if (st != FO_OK) return st;
-    // kernel parameters are copied at launch, so one block of host memory
-    // per thread serves every launch
-    thread_local fo::StepParams P;
     int i = 0;
     while (i < n) {
-        std::memset(&P, 0, offsetof(fo::StepParams, t));
-        P.sc = sc;
-        int m = 0;
-        int64_t chunks = 0;
-        P.chunk_start[0] = 0;
-        for (; i < n && m < fo::kMaxTensorsPerLaunch; i++) {
-            const fo_tensor& x = t[i];
-            if (x.numel == 0) continue;
-            fo::TensorDesc& d = P.t[m];
-            d.w = x.w;
-            d.ecc = x.ecc;
-            d.grad = x.grad;
-            d.mq = x.m_q;
-            d.ms = x.m_scale;
-            d.vq = x.v_q;
-            d.vs = x.v_scale;
-            d.numel = x.numel;
-            // staged chunks: every array 16-byte aligned (bulk copies, 128-bit
-            // stores) and the arrays written with 256-bit stores (weights, 16-bit
-            // ECC codes, with 16 elements per lane) 32-byte aligned; other
-            // tensors take the scalar path
-            const uintptr_t a = (uintptr_t)x.w | (uintptr_t)x.grad | (uintptr_t)x.ecc | (uintptr_t)x.m_q |
-                                (uintptr_t)x.m_scale | (uintptr_t)x.v_q | (uintptr_t)x.v_scale;
-            const uintptr_t a32 = L.lane == 16 ? ((uintptr_t)x.w | (L.ecc_bits == 16 ? (uintptr_t)x.ecc : 0)) : 0;
-            d.n_chunks = (int32_t)((x.numel + chunk - 1) / chunk);
-            d.staged = ((a & 15u) == 0 && (a32 & 31u) == 0) ? 1 : 0;
-            const int64_t last = x.numel - (int64_t)(d.n_chunks - 1) * chunk;  // elements of the last chunk
-            d.last_slices = (int16_t)(last / (32 * L.lane));
-            chunks += d.n_chunks;
-            P.chunk_start[++m] = chunks;
-        }
-        if (m == 0) break;
-        P.n_tensors = m;
-        P.total_chunks = chunks;
-        // a sentinel past the last tensor keeps the device-side walk bounded
-        for (int j = m + 1; j <= fo::kMaxTensorsPerLaunch; j++) P.chunk_start[j] = INT64_MAX;
-        int64_t grid = (chunks + warps - 1) / warps;
-        const int64_t cap = (int64_t)sms * bps;
-        if (grid > cap) grid = cap;
-        L.k<<<(unsigned)grid, L.threads, L.smem, stream>>>(P);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return cuda_fail(e, "step kernel launch");
+        st = launch_table<fo::kMaxTensorsPerLaunch>(L.k, L, sc, t, n, i, (int64_t)sms * bps, stream);
+        if (st != FO_OK) return st;
     }
     return FO_OK;
 }

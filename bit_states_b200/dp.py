@@ -134,12 +134,31 @@ class ShardedState:
                            sl(self.v_q, o, n), sl(self.v_scale, go, ng))
 
 
+def _descriptor_cache():
+    """Descriptors of (state, grad) pairs built once: a bucket's slices do not
+    move between steps, so each step reuses its ctypes descriptor."""
+    from . import fo
+
+    cache = {}
+
+    def get(state, grad):
+        key = (state.w.data_ptr(), state.ecc.data_ptr(), grad.data_ptr(), state.numel)
+        d = cache.get(key)
+        if d is None:
+            d = cache[key] = fo.descriptors([state], [grad])
+        return d
+
+    return get
+
+
 def _adamw_step_fn(fmt, hp):
     from . import fo
 
+    desc = _descriptor_cache()
+
     def step(state, grad, t, stream):
         h = fo.fo_adamw_hparams(hp["lr"], hp["beta1"], hp["beta2"], hp["eps"], hp["weight_decay"], t)
-        fo.fo_adamw_step(fo.descriptors([state], [grad]), 1, fmt, h, stream)
+        fo.fo_adamw_step(desc(state, grad), 1, fmt, h, stream)
 
     return step
 
@@ -147,10 +166,12 @@ def _adamw_step_fn(fmt, hp):
 def _sgdm_step_fn(fmt, hp):
     from . import fo
 
+    desc = _descriptor_cache()
+
     def step(state, grad, t, stream):
         h = fo.fo_sgdm_hparams(hp["lr"], hp["momentum"], hp.get("dampening", 0.0), hp.get("weight_decay", 0.0),
                                int(bool(hp.get("nesterov", False))), t)
-        fo.fo_sgdm_step(fo.descriptors([state], [grad]), 1, fmt, h, stream)
+        fo.fo_sgdm_step(desc(state, grad), 1, fmt, h, stream)
 
     return step
 
@@ -194,6 +215,57 @@ class DataParallelStep:
         self.comm = torch.cuda.Stream(device=dev) if self.cuda else None
         # this rank's reduced gradient, laid out like its owned state arrays
         self.gown = torch.zeros(state.m_q.numel(), dtype=torch.int16, device=dev)
+        self._buckets = None
+
+    def _parts(self):
+        st, L = self.state, self.layout
+        parts = []
+        for bi, b in enumerate(L.buckets):
+            e0 = b.g0 * GROUP
+            s0, s1, go = st.slices[bi]
+            parts.append((e0, e0 + b.groups * GROUP, s0, s1, go * GROUP, (s1 - s0)))
+        return parts
+
+    def exchange(self, grads_flat):
+        """The collectives of one step without the step itself: every bucket's
+        reduce-scatter into this rank's gradient shard, then every bucket's
+        all-gather of x' (unchanged), on the communication stream.  Used to
+        time the exchange alone; the state is left as it was."""
+        import torch
+        import torch.distributed as dist
+
+        gflat = grads_flat.view(self.gdt)
+        wflat = self.state.w.view(self.wdt)
+        parts = self._parts()
+        if not self.cuda:
+            for e0, e1, s0, s1, o, n in parts:
+                dist.reduce_scatter_tensor(self.gown[o:o + n].view(self.gdt), gflat[e0:e1], op=self.op,
+                                           group=self.group)
+                dist.all_gather_into_tensor(wflat[e0:e1], wflat[s0:s1].clone(), group=self.group)
+            return
+        cur = torch.cuda.current_stream()
+        self.comm.wait_stream(cur)
+        with torch.cuda.stream(self.comm):
+            for e0, e1, s0, s1, o, n in parts:
+                dist.reduce_scatter_tensor(self.gown[o:o + n].view(self.gdt), gflat[e0:e1], op=self.op,
+                                           group=self.group)
+            for e0, e1, s0, s1, o, n in parts:
+                dist.all_gather_into_tensor(wflat[e0:e1], wflat[s0:s1], group=self.group)
+        cur.wait_stream(self.comm)
+
+    def _bucket(self, bi: int):
+        """(state of this rank's slice of bucket bi, its gradient shard), views
+        built once."""
+        if self._buckets is None:
+            self._buckets = [(self.state.bucket_state(i), self.gown[o:o + n])
+                             for i, (e0, e1, s0, s1, o, n) in enumerate(self._parts())]
+        return self._buckets[bi]
+
+    def step_only(self, t: int, stream=None):
+        """The fused step of every owned bucket slice on the gradient shard of
+        the last exchange, without collectives (to time the steps alone)."""
+        for bi in range(len(self.layout.buckets)):
+            self.step_fn(*self._bucket(bi), t, stream)
 
     def step(self, grads_flat, t: int):
         """grads_flat: this rank's whole 16-bit gradient in the flat layout
@@ -207,19 +279,15 @@ class DataParallelStep:
         import torch
         import torch.distributed as dist
 
-        st, L = self.state, self.layout
+        st = self.state
         gflat = grads_flat.view(self.gdt)
         wflat = st.w.view(self.wdt)
-        parts = []
-        for bi, b in enumerate(L.buckets):
-            e0 = b.g0 * GROUP
-            s0, s1, go = st.slices[bi]
-            parts.append((e0, e0 + b.groups * GROUP, s0, s1, go * GROUP, (s1 - s0)))
+        parts = self._parts()
         if not self.cuda:
             for bi, (e0, e1, s0, s1, o, n) in enumerate(parts):
                 dist.reduce_scatter_tensor(self.gown[o:o + n].view(self.gdt), gflat[e0:e1], op=self.op,
                                            group=self.group)
-                self.step_fn(st.bucket_state(bi), self.gown[o:o + n], t, None)
+                self.step_fn(*self._bucket(bi), t, None)
                 dist.all_gather_into_tensor(wflat[e0:e1], wflat[s0:s1].clone(), group=self.group)
             return
         cur = torch.cuda.current_stream()
@@ -234,7 +302,7 @@ class DataParallelStep:
                 rs_done.append(ev)
         for bi, (e0, e1, s0, s1, o, n) in enumerate(parts):
             cur.wait_event(rs_done[bi])
-            self.step_fn(st.bucket_state(bi), self.gown[o:o + n], t, cur)
+            self.step_fn(*self._bucket(bi), t, cur)
             ev = torch.cuda.Event()
             ev.record(cur)
             step_done.append(ev)

@@ -312,3 +312,62 @@ def test_layout_properties_random_lists():
         assert 0 <= L.groups - off // GROUP < world
 
     check()
+
+
+# ---- the exchange and the steps alone (what bench.py times separately) ---------------
+
+def _split_worker(rank, world, port, q):
+    import torch
+    import torch.distributed as dist
+
+    import oracle
+    from bit_states_b200.dp import DataParallelStep, ShardedState
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        layout = FlatLayout(NUMELS, world, bucket_groups=BUCKET_GROUPS)
+        w, e = zip(*[oracle.encode_master(_masters(ti, n)) for ti, n in enumerate(NUMELS)])
+        wf, ef = _flat(layout, w, np.uint16), _flat(layout, e, np.int8)
+        states = []
+        for _ in range(2):
+            st = ShardedState(layout, rank, "cpu")
+            st.w.copy_(torch.from_numpy(wf.view(np.int16)))
+            for s0, s1, go in st.slices:
+                st.ecc[go * GROUP:go * GROUP + (s1 - s0)] = torch.from_numpy(ef[s0:s1])
+            states.append(st)
+        a = DataParallelStep(states[0], step_fn=_oracle_step_fn, reduce_op="sum")
+        b = DataParallelStep(states[1], step_fn=_oracle_step_fn, reduce_op="sum")
+        g = torch.from_numpy(_flat(layout, [_grads(rank, ti, 1, n) for ti, n in enumerate(NUMELS)],
+                                   np.uint16).view(np.int16))
+        a.step(g, 1)
+        w_before = states[1].w.clone()
+        b.exchange(g)
+        same_w = bool(torch.equal(states[1].w, w_before))
+        same_grad = bool(torch.equal(a.gown, b.gown))
+        b.step_only(1)
+        sa, sb = states
+        owned_w = all(torch.equal(sa.w[s0:s1], sb.w[s0:s1]) for s0, s1, go in sa.slices)
+        codes = all(torch.equal(getattr(sa, k), getattr(sb, k)) for k in ("ecc", "m_q", "m_scale", "v_q", "v_scale"))
+        q.put((rank, same_w, same_grad, owned_w, codes))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_exchange_alone_and_steps_alone_compose_to_the_step():
+    """exchange() moves the reduced gradient shards and leaves x' as it was;
+    step_only() on those shards then gives the owned bytes of step()."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_split_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=300) for _ in range(2)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, same_w, same_grad, owned_w, codes in res:
+        assert same_w and same_grad and owned_w and codes, (rank, same_w, same_grad, owned_w, codes)
