@@ -122,14 +122,38 @@ class CompressedAdamW:
         descs = fo.descriptors(self.p.states, grads)
         fo.fo_adamw_step(descs, len(self.p.states), self.fmt, self.hparams(self.t), stream)
 
-    def step_tensor(self, i: int, grad, t: int, stream=None):
+    def start_release(self) -> int:
+        """Gradient release: begin one optimizer step whose tensors are then
+        stepped one by one with step_tensor (all with this step count)."""
+        self.t += 1
+        return self.t
+
+    def step_tensor(self, i: int, grad, t: int = None, stream=None):
         """Gradient release: step tensor i alone (its gradient may be freed
-        once the work on the stream has finished)."""
+        once the work on the stream has finished), with step count t (by
+        default the one start_release began)."""
+        if t is None:
+            if self.t < 1:
+                raise ValueError("call start_release() before step_tensor()")
+            t = self.t
         descs = fo.descriptors([self.p.states[i]], [grad])
         fo.fo_adamw_step(descs, 1, self.fmt, self.hparams(t), stream)
 
+    def state_dict(self) -> dict:
+        """The optimizer's part of a checkpoint: the step count (bias
+        corrections depend on it) and the hyper-parameters; the compressed
+        arrays are CompressedParams.state_dict()."""
+        return {"t": self.t, "hparams": dict(self.hp)}
+
+    def load_state_dict(self, d: dict) -> None:
+        self.t = int(d["t"])
+        self.hp.update(d["hparams"])
+
 
 class CompressedSGDM:
+    """SGD with momentum over a parameter list with fp16/bf16 + ECC masters and
+    an 8-bit companded momentum; ``step`` is one fused kernel launch."""
+
     def __init__(self, params: CompressedParams, lr=0.1, momentum=0.9, dampening=0.0,
                  weight_decay=0.0, nesterov=False, grad_dtype="fp16"):
         self.p = params
@@ -147,3 +171,12 @@ class CompressedSGDM:
         self.t += 1
         descs = fo.descriptors(self.p.states, grads)
         fo.fo_sgdm_step(descs, len(self.p.states), self.fmt, self.hparams(self.t), stream)
+
+    def state_dict(self) -> dict:
+        """The optimizer's part of a checkpoint: the step count (the first
+        step copies the gradient into the momentum) and the hyper-parameters."""
+        return {"t": self.t, "hparams": dict(self.hp)}
+
+    def load_state_dict(self, d: dict) -> None:
+        self.t = int(d["t"])
+        self.hp.update(d["hparams"])

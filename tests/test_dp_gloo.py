@@ -9,6 +9,7 @@ import os
 import socket
 
 import numpy as np
+import pytest
 import torch.multiprocessing as mp
 
 from bit_states_b200.dp import GROUP, FlatLayout
@@ -284,8 +285,8 @@ def test_layout_properties_random_lists():
     groups lie inside the layout, buckets tile the groups in order with sizes
     that are multiples of the world size, and every rank's slices are equal,
     disjoint and together cover every group exactly once."""
-    from hypothesis import given, settings
-    from hypothesis import strategies as hs
+    hypothesis = pytest.importorskip("hypothesis")
+    given, settings, hs = hypothesis.given, hypothesis.settings, hypothesis.strategies
 
     @settings(max_examples=200, deadline=None)
     @given(hs.lists(hs.integers(0, 5000), min_size=1, max_size=12), hs.integers(1, 8), hs.integers(1, 300))
