@@ -231,6 +231,36 @@ __global__ void k_rcp_scaling(unsigned long long* cnt, uint32_t* ex)
     }
 }
 
+// The step kernel's bounded wait on an mbarrier (one block of 64 threads):
+// warp 0 waits on a barrier nothing ever arrives on, with a limit of
+// limit_ns; warp 1 waits on a barrier its lane 0 completed by arriving.
+// cnt[0]: threads of warp 0 whose wait did not give up; cnt[1]: threads of
+// warp 1 whose wait gave up; cnt[2]: the longest wait of warp 0 in ns;
+// cnt[3]: the shortest.
+__global__ void k_wait(unsigned long long limit_ns, unsigned long long* cnt)
+{
+    __shared__ __align__(8) uint64_t bars[2];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t bar = (uint32_t)__cvta_generic_to_shared(&bars[warp]);
+    if (lane == 0) {
+        fo::mbar_init(bar, 1);
+        fo::mbar_init_fence();
+    }
+    __syncthreads();
+    if (warp == 1 && lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+    __syncwarp();
+    const unsigned long long t0 = fo::globaltimer();
+    const bool done = fo::mbar_wait_bounded(bar, 0u, limit_ns);
+    const unsigned long long dt = fo::globaltimer() - t0;
+    if (warp == 0) {
+        if (done) atomicAdd(&cnt[0], 1ull);
+        atomicMax(&cnt[2], dt);
+        atomicMin(&cnt[3], dt);
+    } else if (!done) {
+        atomicAdd(&cnt[1], 1ull);
+    }
+}
+
 int launch_done(unsigned long long* hcnt, uint32_t* hex, unsigned long long* dcnt, uint32_t* dex)
 {
     if (cudaGetLastError() != cudaSuccess) return 2;
@@ -245,7 +275,8 @@ int launch_done(unsigned long long* hcnt, uint32_t* hex, unsigned long long* dcn
 // which: 0 ftz forms, 1 square root, 2 division (n pairs, seed), 3 rcp bound
 // and scale reciprocals, 4 / 5 fast bf16 / fp16 ECC8 codec, 6 division over
 // the significand grid (n divisor significands from seed), 7 power-of-two
-// scaling of the approximate reciprocal and reciprocal square root.  cnt: 4 counters, ex: 16 example words (host memory).
+// scaling of the approximate reciprocal and reciprocal square root, 8 the
+// bounded mbarrier wait (n = its limit in ns).  cnt: 4 counters, ex: 16 example words (host memory).
 extern "C" __attribute__((visibility("default"))) int fo_arith_check(int which, uint64_t n, uint64_t seed,
                                                                      unsigned long long* cnt, uint32_t* ex)
 {
@@ -277,6 +308,18 @@ extern "C" __attribute__((visibility("default"))) int fo_arith_check(int which, 
         k_div_grid<<<grid, block>>>((uint32_t)seed, (uint32_t)n, dcnt, dex);
         break;
     case 7: k_rcp_scaling<<<grid, block>>>(dcnt, dex); break;
+    case 8: {
+        // n: the wait limit in ns (at most 1 s); cnt[3] starts at its maximum
+        if (n == 0 || n > 1000000000ull) {
+            cudaFree(dcnt);
+            cudaFree(dex);
+            return 5;
+        }
+        const unsigned long long big = ~0ull;
+        cudaMemcpy(dcnt + 3, &big, sizeof big, cudaMemcpyHostToDevice);
+        k_wait<<<1, 64>>>(n, dcnt);
+        break;
+    }
     default: break;
     }
     const int rc = launch_done(cnt, ex, dcnt, dex);

@@ -18,6 +18,9 @@ the IEEE operations of the exact path):
   two over the exponents the divider's range reaches: every correctly
   rounded step of the divider then commutes with the scaling while its
   intermediates stay normal, which extends the grid to the stated range;
+* the bounded wait on an mbarrier gives up after its limit on a barrier that
+  nothing completes (and returns at once on one that completed), so a staged
+  copy that never lands cannot hang the step kernel;
 * the fast ECC8 codec of 16-bit masters (bit arithmetic; for fp16 an exact
   fma at and below the smallest normal) equals the exact codec: decode of
   every finite 16-bit pattern with every code, encode of every binary32 below
@@ -90,3 +93,10 @@ def test_newton_raphson_quotient_every_significand_pair():
             first = [hex(v) for v in ex[:4]]
     assert total == 0, f"quotient differs on {total} significand pairs, e.g. (x, b) = {first}"
 
+
+def test_bounded_wait_gives_up_on_a_barrier_nothing_completes():
+    limit = 20_000_000  # 20 ms
+    cnt, ex = arith_check.run(8, n=limit)
+    assert cnt[0] == 0, f"{cnt[0]} waits on a barrier nothing completes returned success"
+    assert cnt[1] == 0, f"{cnt[1]} waits on a completed barrier gave up"
+    assert limit <= cnt[3] <= cnt[2] < 1_000_000_000, f"waits lasted {cnt[3]} .. {cnt[2]} ns for a {limit} ns limit"
