@@ -346,6 +346,24 @@ def test_gpt2_small_101_steps_sampled():
             _sampled_check(wl, P, orcs, f"step {t}")
 
 
+def test_gpt2_small_sgdm_sampled():
+    """The GPT-2-small list stepped by SGD-momentum (fp16 + 8-bit ECC, the
+    profiling case for SGD-momentum at a size ten times the L2): 4 sampled
+    groups per tensor (plus the first and last) against the oracle after
+    steps 1 and 2."""
+    wl = workload("gpt2-small-124M-sgdm")
+    P = U.device_state(wl)
+    G = U.GradArena(P)
+    rng = np.random.default_rng(2)
+    orcs = {ti: U.OracleSample(wl, ti, U.sample_groups(t.numel, 4, rng)) for ti, t in enumerate(wl.tensors)}
+    for t in (1, 2):
+        G.fill(wl, t)
+        U.step(wl, P, G, t)
+        for o in orcs.values():
+            o.step(t)
+        _sampled_check(wl, P, orcs, f"step {t}")
+
+
 def test_resnet50_sgdm_every_byte():
     wl = workload("resnet50-25.6M")
     _run_full_compare(wl, 2)

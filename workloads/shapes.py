@@ -114,6 +114,18 @@ def gpt2_small() -> Workload:
                     "one multi-tensor AdamW step after 100 warm steps")
 
 
+def gpt2_small_sgdm() -> Workload:
+    """The GPT-2-small parameter list stepped by SGD-momentum with fp16 + 8-bit
+    ECC masters (the ResNet-50 recipe's optimizer and formats): an SGD-momentum
+    case whose 1.26 GB per step is ten times the L2, for profiler captures."""
+    w = gpt2_small()
+    return Workload(
+        name="gpt2-small-124M-sgdm", tensors=w.tensors, optimizer="sgdm", hparams=dict(SGDM_HP),
+        w_dtype="fp16", grad_dtype="fp16", grad_dist="normal", grad_scale=1e-2, warm_steps=1,
+        description="GPT-2-small parameter list (148 tensors), fp16 + 8-bit ECC masters, "
+                    "SGD momentum 0.9")
+
+
 def _conv(name, cout, cin, k):
     return TensorSpec(name, (cout, cin, k, k), "normal", math.sqrt(2.0 / (cin * k * k)))
 
@@ -196,6 +208,7 @@ def llama31_layers(n_layers: int = 2) -> Workload:
 CONFIGS = {
     "flat-1M": flat_1m,
     "gpt2-small-124M": gpt2_small,
+    "gpt2-small-124M-sgdm": gpt2_small_sgdm,
     "resnet50-25.6M": resnet50,
     "llama3.1-8b": llama31_8b,
     "llama3.1-8b-2layers": llama31_layers,
