@@ -386,26 +386,39 @@ def main():
     sampler.start()
 
     K = args.steps
-    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev) if args.flush_l2 else None
+    # one event pair around the K steps; with an L2 flush between steps, one
+    # pair per step, so that only the steps themselves are timed (events
+    # between steps would add host work per step, which shows on lists whose
+    # step takes tens of microseconds)
+    nev = K if flush is not None else 1
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(nev)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(nev)]
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
+    if flush is None:
+        ev_s[0].record(stream)
     for k in range(K):
         t += 1
         if flush is not None:
             flush.fill_(k & 0xFF)
-        ev_s[k].record(stream)
+            ev_s[k].record(stream)
         do_step(t)
-        ev_e[k].record(stream)
+        if flush is not None:
+            ev_e[k].record(stream)
+    if flush is None:
+        ev_e[0].record(stream)
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     clocks = sampler.stop()
-    per_launch_ms = statistics.mean(ev_s[k].elapsed_time(ev_e[k]) for k in range(K))
-    # with an L2 flush between steps only the steps themselves are timed
-    total_ms = per_launch_ms * K if flush is not None else ev_s[0].elapsed_time(ev_e[K - 1])
+    if flush is not None:
+        per_launch_ms = statistics.mean(ev_s[k].elapsed_time(ev_e[k]) for k in range(K))
+        total_ms = per_launch_ms * K
+    else:
+        total_ms = ev_s[0].elapsed_time(ev_e[0])
+        per_launch_ms = total_ms / K
     if dist:
         tt = torch.tensor([total_ms, per_launch_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
