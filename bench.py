@@ -35,6 +35,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "fused AdamW step Gparams/s and achieved HBM GB/s vs B200 peak"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e specification (context beside the measured or fallback peak)
 
 
 def parse():
@@ -515,8 +516,8 @@ def main():
             "config": arm_config(wl, args, world),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic,
-                         "peak_kind": peak_kind, "algorithmic_bytes_per_launch": abytes,
-                         "kernel": "fo::step_kernel"},
+                         "peak_kind": peak_kind, "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
+                         "algorithmic_bytes_per_launch": abytes, "kernel": "fo::step_kernel"},
             "ceiling": None if ceiling_ms is None else {
                 "kernel": "fo_stream_copy: the step's byte mix with the same staging, work split and "
                           "stores, no arithmetic (after the timed region)",
@@ -710,6 +711,7 @@ def run_dp(args, rank, world, local):
                                             "all_gather_in": 2 * layout.numel * (world - 1) // world}},
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": None, "peak_kind": peak_kind,
+                         "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
                          "algorithmic_bytes_per_launch": int(step_bytes / max(1, len(layout.buckets))),
                          "kernel": "fo::step_kernel (the owned slices' steps, timed without the exchange)"},
             "clocks": clocks,

@@ -108,9 +108,7 @@ __global__ void k_div(uint64_t n, uint64_t seed, unsigned long long* cnt, uint32
 
 // cnt[0]: largest ulp distance of rcp_approx(d) from RN(1/d) over every
 // binary32 d in [1, 2]; cnt[1]: scale_recips(S, S) != (1/S, 255/S) by div.rn
-// for every positive finite fp16 S (and S = 0 must give (0, 0)); cnt[2]:
-// v_code_value2 != RN(q / 255) by div.rn for a code q in [0, 255] (both byte
-// positions of a pair)
+// for every positive finite fp16 S (and S = 0 must give (0, 0))
 __global__ void k_rcp_scales(unsigned long long* cnt, uint32_t* ex)
 {
     const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
@@ -119,18 +117,6 @@ __global__ void k_rcp_scales(unsigned long long* cnt, uint32_t* ex)
         const float r = fo::rcp_approx(d), e = __fdiv_rn(1.0f, d);
         const int u = (int)__float_as_uint(r) - (int)__float_as_uint(e);
         atomicMax(&cnt[0], (unsigned long long)(u < 0 ? -u : u));
-    }
-    for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < 256ull; i += stride) {
-        // both byte positions of a pair: codes i and 255 - i in bytes 2, 3 of the word
-        const uint32_t q0 = (uint32_t)i, q1 = 255u - (uint32_t)i;
-        const float2 v = fo::v_code_value2((q0 << 16) | (q1 << 24), 2u);
-        if (__float_as_uint(v.x) != __float_as_uint(__fdiv_rn((float)q0, 255.0f)) ||
-            __float_as_uint(v.y) != __float_as_uint(__fdiv_rn((float)q1, 255.0f)))
-            note(cnt, ex, 2, (uint32_t)i);
-        const float2 w = fo::v_code_value2(q0 | (q1 << 8), 0u);
-        if (__float_as_uint(w.x) != __float_as_uint(__fdiv_rn((float)q0, 255.0f)) ||
-            __float_as_uint(w.y) != __float_as_uint(__fdiv_rn((float)q1, 255.0f)))
-            note(cnt, ex, 2, (uint32_t)i);
     }
     for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < 0x7C00ull; i += stride) {
         const float S = __half2float(__ushort_as_half((unsigned short)i));
