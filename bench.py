@@ -47,6 +47,10 @@ def parse():
     ap.add_argument("--config", default="llama3.1-8b")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-piece", type=int, default=1 << 26,
+                    help="parameters per host<->device piece of the end-to-end leg (whole groups; 2^26 measured "
+                         "best of 2^23..2^26)")
+    ap.add_argument("--e2e-ring", type=int, default=3, help="device stage buffers of the end-to-end leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-params", type=int, default=1 << 24)
     ap.add_argument("--launch-mode", default="multi", choices=["multi", "release"])
@@ -739,7 +743,7 @@ def run_e2e(args, wl, P, fmt, dev, dist, world, torch, fo):
         return None
     from workloads import device as wdev
 
-    PIECE, RING = 1 << 24, 4
+    PIECE, RING = max(32, args.e2e_piece // 32 * 32), max(2, args.e2e_ring)
     pieces = []                            # (tensor, first element, elements), release order
     for ti in list(range(len(P.numels)))[::-1]:
         n = P.numels[ti]
