@@ -62,8 +62,8 @@
  *   - Results do not depend on the number of tensors per call, their order,
  *     or on whether they are stepped in one call or one call per tensor.
  *   - Launch geometry (performance only, results identical): chunks of 1024
- *     elements (512 where the stage buffers would not fit), staged in shared
- *     memory by bulk copies, one warp per chunk; the elements of a tensor's
+ *     elements for AdamW and 512 for SGD-momentum, staged in shared memory by
+ *     bulk copies, one warp per chunk; the elements of a tensor's
  *     last chunk beyond its whole 512-element slices, and tensors whose
  *     arrays are not 16-byte aligned (or whose weights / 16-bit ECC codes are
  *     not 32-byte aligned), take a scalar path.
