@@ -418,6 +418,7 @@ def main():
     if dist:
         dist.barrier()
     clocks = sampler.stop()
+    fo.fo_check_errors()  # raises if a step kernel gave up a bounded wait (chunks left unstepped)
     if flush is not None:
         per_launch_ms = statistics.mean(ev_s[k].elapsed_time(ev_e[k]) for k in range(K))
         total_ms = per_launch_ms * K
