@@ -139,6 +139,10 @@ __global__ void k_rcp_scales(unsigned long long* cnt, uint32_t* ex)
 template <int W>
 __global__ void k_codec(unsigned long long* cnt, uint32_t* ex)
 {
+    // The fp16 fast codec takes a warp vote, so every call below is made by
+    // whole warps: the stride and both loop bounds are multiples of 32, and
+    // the 32 consecutive items of a warp share one pattern h (128 items per h),
+    // so a warp skips a non-finite h together.
     const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
     for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (1ull << 16) * 128ull; i += stride) {
         const uint32_t h = (uint32_t)(i >> 7), k = (uint32_t)(i & 127u);
