@@ -41,7 +41,8 @@
  * Conventions for every call:
  *   - Memory: the caller owns every buffer; the library allocates nothing and
  *     keeps no state between calls other than per-device launch constants
- *     (SM count), found on the first call on a device.
+ *     (SM count), found on the first call on a device, and a device word that
+ *     counts bounded waits that gave up (read and cleared by fo_check_errors).
  *   - Asynchrony: work is enqueued on `stream` (a cudaStream_t; NULL is the
  *     legacy default stream) and the call returns without waiting.  The
  *     descriptor array and hyper-parameter structs are copied into the launch
