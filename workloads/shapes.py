@@ -192,7 +192,7 @@ def llama31_8b(order: str = "forward", ecc_bits: int = 8) -> Workload:
     return wl
 
 
-def llama31_layers(n_layers: int = 2) -> Workload:
+def llama31_layers(n_layers: int = 2, ecc_bits: int = 8) -> Workload:
     """The first decoder layers of the Llama-3.1-8B list (same shapes, values
     and hyper-parameters as in the full list): a case of a few GB, far above
     the L2, for profiler captures of the full-size kernel."""
@@ -200,9 +200,10 @@ def llama31_layers(n_layers: int = 2) -> Workload:
     per_layer = 9
     ts = full.tensors[1:1 + per_layer * n_layers]
     return Workload(
-        name=f"llama3.1-8b-{n_layers}layers", tensors=ts, optimizer="adamw", hparams=dict(ADAMW_HP),
-        grad_dist="student_t3", grad_scale=1e-4, warm_steps=0,
-        description=f"decoder layers 0..{n_layers - 1} of the Llama-3.1-8B parameter list")
+        name=f"llama3.1-8b-{n_layers}layers" + ("" if ecc_bits == 8 else "-ecc16"), tensors=ts, optimizer="adamw",
+        hparams=dict(ADAMW_HP), ecc_bits=ecc_bits, grad_dist="student_t3", grad_scale=1e-4, warm_steps=0,
+        description=f"decoder layers 0..{n_layers - 1} of the Llama-3.1-8B parameter list"
+                    + ("" if ecc_bits == 8 else ", 16-bit ECC"))
 
 
 CONFIGS = {
@@ -220,4 +221,6 @@ def workload(name: str) -> Workload:
         return llama31_8b("release")
     if name == "llama3.1-8b-ecc16":
         return llama31_8b(ecc_bits=16)
+    if name == "llama3.1-8b-2layers-ecc16":
+        return llama31_layers(2, ecc_bits=16)
     return CONFIGS[name]()
